@@ -1,0 +1,164 @@
+"""CPU oracle for the N:M sparse weight x dense activation GEMM -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never does, and this
+package imports nothing from the product library: the two share no code.
+
+What it computes follows "Realizable N:M Sparse Transformer Inference via
+Search-Kernel Co-Design" (arXiv 2607.12505):
+
+* section 2.1 -- N:M sparsity: every group of M weights keeps N non-zeros;
+* section 4.2 -- micro-dense execution materialises only those N values per
+  window and runs dense MMA on them, so the product equals the dense GEMM over
+  the masked weight; the packed format carries values and in-window positions.
+
+The arithmetic lives in ``nm_oracle.c`` (plain C, one OpenMP loop over output
+rows, ``-ffp-contract=off``).  This module only builds it, marshals numpy
+arrays, and states the readings of the paper that the C code follows:
+
+* groups run along K, contiguous, aligned at k = 0;
+* top-N by magnitude, ties to the lower in-group position;
+* exactly N slots per group, kept values in ascending position;
+* ``idx`` holds one 4-bit position per kept element, two per byte, low nibble
+  first, each row padded to whole bytes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nm_oracle.c")
+_LIB = os.path.join(_HERE, "libnm_oracle.so")
+
+DTYPES = {"int8": 0, "fp16": 1, "bf16": 2}
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``nm_oracle.c`` into ``libnm_oracle.so`` next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared",
+             "-std=c11", "-Wall", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i64, p, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+        lib.oracle_compress.argtypes = [p, i64, i64, i32, i32, i32, p, p]
+        lib.oracle_decompress.argtypes = [p, p, i64, i64, i32, i32, i32, p]
+        lib.oracle_gemm_i8.argtypes = [p, i64, i64, p, i64, p, p, p]
+        lib.oracle_gemm_f16.argtypes = [p, i64, i64, p, i64, i32, p, p]
+        lib.oracle_idx_pitch.argtypes = [i64, i32, i32]
+        lib.oracle_idx_pitch.restype = i64
+        lib.oracle_threads.restype = i32
+        lib.oracle_set_threads.argtypes = [i32]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _dtype_code(a: np.ndarray, dtype: str | None) -> int:
+    if dtype is None:
+        if a.dtype == np.int8:
+            dtype = "int8"
+        elif a.dtype == np.float16:
+            dtype = "fp16"
+        else:
+            raise ValueError("pass dtype='bf16' for raw uint16 bfloat16 bits")
+    return DTYPES[dtype]
+
+
+def threads() -> int:
+    return _load().oracle_threads()
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def idx_pitch(k: int, N: int, M: int) -> int:
+    return int(_load().oracle_idx_pitch(k, N, M))
+
+
+def compress(W: np.ndarray, N: int, M: int, dtype: str | None = None):
+    """Top-N-of-M compression of W [n_out, k] along k.
+
+    ``W`` is int8, float16, or uint16 holding bfloat16 bits (``dtype='bf16'``).
+    Returns ``(values [n_out, k//M, N], idx [n_out, idx_pitch] uint8)``.
+    """
+    W = np.ascontiguousarray(W)
+    n_out, k = W.shape
+    code = _dtype_code(W, dtype)
+    values = np.zeros((n_out, k // M, N), dtype=W.dtype)
+    idx = np.zeros((n_out, idx_pitch(k, N, M)), dtype=np.uint8)
+    rc = _load().oracle_compress(_ptr(W), n_out, k, code, N, M, _ptr(values), _ptr(idx))
+    if rc != 0:
+        raise ValueError(f"oracle_compress rejected the arguments (rc={rc})")
+    return values, idx
+
+
+def decompress(values: np.ndarray, idx: np.ndarray, n_out: int, k: int, N: int, M: int,
+               dtype: str | None = None) -> np.ndarray:
+    """Scatter the kept values back into a dense masked W [n_out, k]."""
+    values = np.ascontiguousarray(values)
+    idx = np.ascontiguousarray(idx, dtype=np.uint8)
+    code = _dtype_code(values, dtype)
+    Wm = np.zeros((n_out, k), dtype=values.dtype)
+    rc = _load().oracle_decompress(_ptr(values), _ptr(idx), n_out, k, code, N, M, _ptr(Wm))
+    if rc != 0:
+        raise ValueError(f"oracle_decompress rejected the arguments (rc={rc})")
+    return Wm
+
+
+def gemm(X: np.ndarray, Wm: np.ndarray, scale: np.ndarray | None = None,
+         dtype: str | None = None) -> np.ndarray:
+    """Y = X @ Wm.T over the masked weight.
+
+    int8 inputs: int32 result, or float32 ``(float)acc * scale[n]`` when
+    ``scale`` is given.  fp16/bf16 inputs: float64 result (times ``scale``).
+    """
+    X = np.ascontiguousarray(X)
+    Wm = np.ascontiguousarray(Wm)
+    T, K = X.shape
+    n_out, K2 = Wm.shape
+    if K != K2:
+        raise ValueError("K mismatch")
+    code = _dtype_code(X, dtype)
+    lib = _load()
+    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.float32)
+    sp = None if sc is None else _ptr(sc)
+    if code == 0:
+        if sc is None:
+            Y = np.zeros((T, n_out), dtype=np.int32)
+            rc = lib.oracle_gemm_i8(_ptr(X), T, K, _ptr(Wm), n_out, None, _ptr(Y), None)
+        else:
+            Y = np.zeros((T, n_out), dtype=np.float32)
+            rc = lib.oracle_gemm_i8(_ptr(X), T, K, _ptr(Wm), n_out, sp, None, _ptr(Y))
+    else:
+        Y = np.zeros((T, n_out), dtype=np.float64)
+        rc = lib.oracle_gemm_f16(_ptr(X), T, K, _ptr(Wm), n_out, code, sp, _ptr(Y))
+    if rc != 0:
+        raise ValueError(f"oracle gemm failed (rc={rc})")
+    return Y
+
+
+def spmm(X: np.ndarray, W: np.ndarray, N: int, M: int, scale: np.ndarray | None = None,
+         dtype: str | None = None) -> np.ndarray:
+    """The whole path: compress W, decompress, dense GEMM over the masked W."""
+    values, idx = compress(W, N, M, dtype)
+    Wm = decompress(values, idx, W.shape[0], W.shape[1], N, M, dtype)
+    return gemm(X, Wm, scale, dtype)

@@ -1,0 +1,218 @@
+/*
+ * nm_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, obviously-correct CPU statement of what the N:M sparse GEMM
+ * path computes.  Only the test-suite, the smoke check and the CPU-baseline leg
+ * of the benchmark may load it.  It shares no source with the CUDA library.
+ *
+ * Source: "Realizable N:M Sparse Transformer Inference via Search-Kernel
+ * Co-Design" (arXiv 2607.12505).
+ *   - section 2.1: N:M sparsity keeps N non-zeros in every group of M weights.
+ *   - section 4.2: the micro-dense kernel materialises exactly those N values
+ *     per window and runs regular dense MMA fragments on them, so its result is
+ *     the dense GEMM over the masked weight.  The packed format carries the
+ *     values and their positions inside each window.
+ * Readings where the paper is silent (all listed in the design notes):
+ *   - groups run along K (the reduction axis), contiguous, aligned at k = 0;
+ *   - selection is by magnitude, ties go to the lower in-group position;
+ *   - exactly N slots are stored per group (zeros are chosen by the same rule);
+ *   - kept values are stored in ascending in-group position.
+ *
+ * Arithmetic:
+ *   - INT8 GEMM: exact int64 accumulation, then checked to fit int32;
+ *   - INT8 scaled: (float)acc rounded to nearest, then one fp32 multiply
+ *     (build with -ffp-contract=off);
+ *   - FP16/BF16 GEMM: inputs decoded exactly to double, fp64 accumulation,
+ *     result returned in fp64.
+ *
+ * Parity pins (tests/test_oracle.py): hand-worked 4x8 examples, brute-force
+ * subset enumeration, invariants, and exact integer matmul cross-checks.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_INT8 = 0, OR_FP16 = 1, OR_BF16 = 2 };
+
+/* ---- exact decoders for the 16-bit float formats (IEEE binary16, bfloat16) */
+
+static double fp16_to_double(uint16_t h) {
+    int sign = h >> 15;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);                 /* subnormal: m * 2^-24 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(m | 0x400), e - 25);    /* (1.m) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+static double bf16_to_double(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static size_t elem_size(int dtype) { return dtype == OR_INT8 ? 1 : 2; }
+
+/* |w| of element i as a double (exact for all three formats). */
+static double magnitude(const void *w, int dtype, int64_t i) {
+    if (dtype == OR_INT8) return fabs((double)((const int8_t *)w)[i]);
+    uint16_t h = ((const uint16_t *)w)[i];
+    return fabs(dtype == OR_FP16 ? fp16_to_double(h) : bf16_to_double(h));
+}
+
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* Bytes of the 4-bit index stream of one row: one nibble per kept element,
+ * two per byte, low nibble first; a row with an odd count ends in a zero
+ * high nibble so that rows never share a byte. */
+int64_t oracle_idx_pitch(int64_t k, int N, int M) {
+    int64_t kept = (k / M) * N;
+    return (kept + 1) / 2;
+}
+
+/*
+ * Compress: for every row r and every group g of M consecutive K positions,
+ * position p is kept iff fewer than N positions q of the same group precede it
+ * in the order (|w| descending, position ascending).  That is the top-N rule
+ * with ties to the lower index, written as a rank test.  Kept positions come
+ * out in ascending order because p is scanned upward.
+ *
+ * values: [n_out][k/M][N] elements of the weight dtype.
+ * idx:    [n_out][idx_pitch] bytes; element e of a row sits in byte e/2,
+ *         low nibble when e is even.
+ * Returns 0, or -1 for an invalid argument.
+ */
+int oracle_compress(const void *W, int64_t n_out, int64_t k, int dtype, int N, int M,
+                    void *values, uint8_t *idx) {
+    if (!W || !values || !idx || n_out <= 0 || k <= 0 || M <= 0 || M > 16 || N <= 0 ||
+        N > M || k % M != 0 || dtype < 0 || dtype > 2)
+        return -1;
+    const size_t es = elem_size(dtype);
+    const int64_t groups = k / M;
+    const int64_t pitch = oracle_idx_pitch(k, N, M);
+    memset(idx, 0, (size_t)(n_out * pitch));
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_out; ++r) {
+        int64_t e = 0; /* kept-element counter within the row */
+        for (int64_t g = 0; g < groups; ++g) {
+            const int64_t base = r * k + g * M;
+            for (int p = 0; p < M; ++p) {
+                double ap = magnitude(W, dtype, base + p);
+                int ahead = 0;
+                for (int q = 0; q < M; ++q) {
+                    double aq = magnitude(W, dtype, base + q);
+                    if (aq > ap || (aq == ap && q < p)) ++ahead;
+                }
+                if (ahead < N) {
+                    memcpy((char *)values + (size_t)(r * groups * N + e) * es,
+                           (const char *)W + (size_t)(base + p) * es, es);
+                    uint8_t *byte = idx + r * pitch + e / 2;
+                    *byte |= (uint8_t)((p & 0xF) << ((e & 1) ? 4 : 0));
+                    ++e;
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/* Decompress: scatter every kept value to its position; all else is zero. */
+int oracle_decompress(const void *values, const uint8_t *idx, int64_t n_out, int64_t k,
+                      int dtype, int N, int M, void *Wm) {
+    if (!values || !idx || !Wm || n_out <= 0 || k <= 0 || M <= 0 || N <= 0 || N > M ||
+        k % M != 0 || dtype < 0 || dtype > 2)
+        return -1;
+    const size_t es = elem_size(dtype);
+    const int64_t groups = k / M;
+    const int64_t pitch = oracle_idx_pitch(k, N, M);
+    memset(Wm, 0, (size_t)(n_out * k) * es);
+    for (int64_t r = 0; r < n_out; ++r) {
+        for (int64_t e = 0; e < groups * N; ++e) {
+            uint8_t byte = idx[r * pitch + e / 2];
+            int p = (e & 1) ? (byte >> 4) : (byte & 0xF);
+            int64_t g = e / N;
+            memcpy((char *)Wm + (size_t)(r * k + g * M + p) * es,
+                   (const char *)values + (size_t)(r * groups * N + e) * es, es);
+        }
+    }
+    return 0;
+}
+
+/*
+ * INT8 GEMM over the masked weight: Y[t][n] = sum_k X[t][k] * Wm[n][k].
+ * Exact int64 accumulation; returns -2 if any result leaves the int32 range
+ * (it cannot for |x| <= 128, |w| <= 128, k <= 131072).
+ * When scale is non-NULL the result is written to Yf as
+ * (float)acc * scale[n] (round-to-nearest conversion, one fp32 multiply);
+ * otherwise to Yi as int32.
+ */
+int oracle_gemm_i8(const int8_t *X, int64_t T, int64_t K, const int8_t *Wm, int64_t n_out,
+                   const float *scale, int32_t *Yi, float *Yf) {
+    if (!X || !Wm || T < 0 || K <= 0 || n_out <= 0 || (!scale && !Yi) || (scale && !Yf))
+        return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t n = 0; n < n_out; ++n) {
+            int64_t acc = 0;
+            for (int64_t kk = 0; kk < K; ++kk)
+                acc += (int64_t)X[t * K + kk] * (int64_t)Wm[n * K + kk];
+            if (acc > INT32_MAX || acc < INT32_MIN) bad = 1;
+            if (scale) {
+                float f = (float)(int32_t)acc;
+                float s = scale[n];
+                volatile float prod = f * s; /* a single rounded fp32 multiply */
+                Yf[t * n_out + n] = prod;
+            } else {
+                Yi[t * n_out + n] = (int32_t)acc;
+            }
+        }
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * FP16/BF16 GEMM over the masked weight, in fp64:
+ * Y[t][n] = (sum_k x(t,k) * w(n,k)) * (scale ? scale[n] : 1), every input
+ * decoded exactly; the result stays in double for the tolerance check.
+ */
+int oracle_gemm_f16(const uint16_t *X, int64_t T, int64_t K, const uint16_t *Wm, int64_t n_out,
+                    int dtype, const float *scale, double *Y) {
+    if (!X || !Wm || !Y || T < 0 || K <= 0 || n_out <= 0 || (dtype != OR_FP16 && dtype != OR_BF16))
+        return -1;
+    double (*dec)(uint16_t) = dtype == OR_FP16 ? fp16_to_double : bf16_to_double;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t n = 0; n < n_out; ++n) {
+            double acc = 0.0;
+            for (int64_t kk = 0; kk < K; ++kk)
+                acc += dec(X[t * K + kk]) * dec(Wm[n * K + kk]);
+            Y[t * n_out + n] = scale ? acc * (double)scale[n] : acc;
+        }
+    }
+    return 0;
+}
