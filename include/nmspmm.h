@@ -1,0 +1,166 @@
+/*
+ * nmspmm.h -- C ABI of the B200 (sm_100a) N:M sparse weight x dense activation
+ * GEMM library (libnmspmm.so).
+ *
+ * The operation is the one of "Realizable N:M Sparse Transformer Inference via
+ * Search-Kernel Co-Design" (arXiv 2607.12505):
+ *   - section 2.1: N:M semi-structured sparsity keeps N non-zeros in every
+ *     group of M weights of the projection and FFN linears;
+ *   - section 4.1: the kernel rests on three mechanisms -- weight packing for
+ *     decode-friendly storage, micro-dense execution, adaptive parallelism;
+ *   - section 4.2: only the N kept values of each window are materialised in
+ *     dense, MMA-shaped tiles; the packed weight carries values and their
+ *     in-window positions together, so no separate index load is needed.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_dev are device pointers of the current CUDA device;
+ *     *_host are host pointers.  The caller owns every buffer it passes.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls are stream-ordered and never synchronise the host unless
+ *     stated.
+ *   - Errors are returned as nm_status, never thrown or trapped; a message for
+ *     the last failing call of the calling thread is in nm_last_error().
+ *   - Layouts are row-major: W [n_out][k] (the PyTorch Linear layout),
+ *     X [T][k], Y [T][n_out].
+ */
+#ifndef NMSPMM_H
+#define NMSPMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NM_OK = 0,
+    NM_ERR_INVALID = 1,     /* bad argument: null pointer, bad size, misalignment */
+    NM_ERR_UNSUPPORTED = 2, /* valid request the library does not implement       */
+    NM_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed                  */
+    NM_ERR_OOM = 4,         /* device allocation failed                           */
+    NM_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (see nm_device_status) */
+} nm_status;
+
+typedef enum { NM_INT8 = 0, NM_FP16 = 1, NM_BF16 = 2 } nm_dtype;
+
+/* Opaque handle holding one compressed weight; owns all device memory it allocates. */
+typedef struct nm_handle nm_handle;
+
+/*
+ * nm_compress -- prune and pack one weight (paper sections 2.1 and 4.2,
+ * "weight packing").
+ *
+ * For every row n and every group g of M consecutive k positions (aligned at
+ * k = 0) keeps the N entries of largest |W|, ties to the lower position, and
+ * builds two device images inside the new handle:
+ *   - the canonical compressed format (see nm_export), and
+ *   - the packed operand image the SpMM kernel streams: per 128-row x k-block
+ *     tile, the kept values already laid out as swizzled tensor-core operand
+ *     rows, followed by their 2-bit in-window positions in the layout the
+ *     sparse tensor core reads.
+ *
+ * W_dev   [n_out][k] of dtype `dt`, 16-byte aligned.  It may be freed once the
+ *         stream has passed this call.
+ * (N, M)  one of (1,4), (2,4), (2,8), (4,8), or N == M with M in {4, 8}
+ *         (dense pass-through).  Other pairs -> NM_ERR_UNSUPPORTED.
+ * k       multiple of M (else NM_ERR_INVALID); n_out, k > 0, at most 2^24.
+ * out     receives the handle; *out is NULL on failure.
+ * Allocates device memory (NM_ERR_OOM on failure); returns without waiting
+ * for the kernels.
+ */
+nm_status nm_compress(const void* W_dev, int64_t n_out, int64_t k, nm_dtype dt, int N, int M,
+                      void* stream, nm_handle** out);
+
+/*
+ * nm_recompress -- prune and pack a new weight of the handle's shape, dtype and
+ * N:M into the handle's existing device buffers (a weight update; same rule
+ * and layouts as nm_compress).  Allocates nothing; stream-ordered, so an
+ * nm_spmm on the same stream afterwards sees the new weight.  W_dev element
+ * aligned, [n_out][k].
+ */
+nm_status nm_recompress(nm_handle* h, const void* W_dev, void* stream);
+
+/*
+ * nm_spmm -- Y = X . Wm^T with Wm the masked weight of `h` (paper section 4.2,
+ * micro-dense execution; section 4.1, adaptive parallelism).
+ *
+ * X_dev     [T][k] of the handle's dtype, 16-byte aligned, k * sizeof(dtype)
+ *           a multiple of 16 bytes (else NM_ERR_UNSUPPORTED).
+ * Y_dev     [T][n_out]:
+ *             INT8, scale_dev == NULL : int32, exact integer result;
+ *             INT8, scale_dev != NULL : float32, (float)acc * scale[n]
+ *                                       (round-to-nearest, one multiply);
+ *             FP16/BF16               : same dtype as X, rounded to nearest
+ *                                       once from the fp32 accumulator
+ *                                       (times scale[n] when given).
+ *           Must be 16-byte aligned and must not overlap X.
+ * scale_dev float32 [n_out] or NULL.
+ * T         >= 0; T == 0 is a no-op returning NM_OK.
+ * The tile shape and split-K factor are chosen per (T, k, n_out, N:M, dtype)
+ * so that small token counts still occupy every SM.  When split-K is used the
+ * handle's workspace is used: calls on one handle must not overlap on the GPU
+ * (the same rule as a library handle with a workspace).  The first call that
+ * needs split-K allocates that workspace (make it before any stream capture).
+ * Never synchronises.
+ */
+nm_status nm_spmm(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
+                  const float* scale_dev, void* stream);
+
+/*
+ * nm_decompress -- write the masked dense weight Wm [n_out][k] (dtype of the
+ * handle) decoded from the packed operand image the SpMM kernel reads, so the
+ * image can be checked against the top-N rule.  W_dev_out 16-byte aligned.
+ */
+nm_status nm_decompress(const nm_handle* h, void* W_dev_out, void* stream);
+
+/*
+ * nm_export -- copy the canonical compressed format to the host.  Synchronises
+ * the device.
+ *   values_host: [n_out][k/M][N] elements of the weight dtype, kept values in
+ *                ascending in-group position (nm_export_sizes gives bytes);
+ *   idx_host:    [n_out][idx_pitch] bytes, one 4-bit in-group position per
+ *                kept element in the same order, two per byte, low nibble
+ *                first; idx_pitch = ceil(N * k / M / 2) so rows never share a
+ *                byte.  For N == M, positions are 0..M-1.
+ */
+nm_status nm_export(const nm_handle* h, void* values_host, uint8_t* idx_host);
+nm_status nm_export_sizes(const nm_handle* h, size_t* values_bytes, size_t* idx_bytes);
+
+/* nm_query -- shape and format of a handle; any output pointer may be NULL. */
+nm_status nm_query(const nm_handle* h, int64_t* n_out, int64_t* k, int* N, int* M, nm_dtype* dt);
+
+/*
+ * nm_device_status -- read (and clear) the handle's device error word, which a
+ * kernel sets instead of trapping when a bounded wait runs out.  Synchronises
+ * the device.  Returns NM_OK or NM_ERR_TIMEOUT.
+ */
+nm_status nm_device_status(const nm_handle* h);
+
+/* nm_destroy -- free the handle and its device memory (synchronises). NULL is a no-op. */
+void nm_destroy(nm_handle* h);
+
+/* nm_last_error -- message of the calling thread's last failing call ("" if none). */
+const char* nm_last_error(void);
+
+/* nm_version -- library version string. */
+const char* nm_version(void);
+
+/*
+ * Test hook (no counterpart in the paper): run nm_spmm with the SpMM kernel's
+ * producer leaving pipeline stage number `skip_stage` (counted over the CTA's
+ * whole run) unfilled, and every bounded wait limited to `timeout_ns`
+ * (0 < timeout_ns <= 2e9).  The MMA warp's wait on that stage then runs out:
+ * the kernel records the timeout in the handle's error word, drains its own
+ * copies and MMAs, frees its tensor memory and returns, so the context stays
+ * usable.  Exists so tests can exercise the failure path without faulting or
+ * hanging a GPU; Y is left partially written.
+ */
+nm_status nm_test_spmm_skip_stage(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
+                                  const float* scale_dev, void* stream, int skip_stage, int64_t timeout_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NMSPMM_H */

@@ -1,1 +1,207 @@
-"""B200-native N:M semi-structured sparse weight x dense activation GEMM."""
+"""B200-native N:M semi-structured sparse weight x dense activation GEMM.
+
+A thin ctypes binding over ``libnmspmm.so`` (C ABI in ``include/nmspmm.h``).
+Every step of the path runs in the library's sm_100a kernels; this module only
+marshals torch tensors (device memory and streams) into the C calls, with the
+same names.  There is no fallback: if the library is missing or a call fails,
+an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnmspmm.so")
+
+NM_OK, NM_ERR_INVALID, NM_ERR_UNSUPPORTED, NM_ERR_CUDA, NM_ERR_OOM, NM_ERR_TIMEOUT = range(6)
+STATUS_NAMES = {0: "NM_OK", 1: "NM_ERR_INVALID", 2: "NM_ERR_UNSUPPORTED", 3: "NM_ERR_CUDA",
+                4: "NM_ERR_OOM", 5: "NM_ERR_TIMEOUT"}
+NM_INT8, NM_FP16, NM_BF16 = 0, 1, 2
+_TORCH_DT = {torch.int8: NM_INT8, torch.float16: NM_FP16, torch.bfloat16: NM_BF16}
+_ELEM = {NM_INT8: torch.int8, NM_FP16: torch.float16, NM_BF16: torch.bfloat16}
+
+# Every symbol include/nmspmm.h declares.
+EXPORTS = ("nm_compress", "nm_recompress", "nm_spmm", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
+           "nm_device_status", "nm_destroy", "nm_last_error", "nm_version", "nm_test_spmm_skip_stage")
+
+
+class NMError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnmspmm.so (built in-tree by ``build.py``); raise if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m structured_sparse_gemm_compress_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.nm_compress.argtypes = [vp, i64, i64, i32, i32, i32, vp, ctypes.POINTER(vp)]
+        L.nm_recompress.argtypes = [vp, vp, vp]
+        L.nm_spmm.argtypes = [vp, vp, i64, vp, vp, vp]
+        L.nm_test_spmm_skip_stage.argtypes = [vp, vp, i64, vp, vp, vp, i32, i64]
+        L.nm_decompress.argtypes = [vp, vp, vp]
+        L.nm_export.argtypes = [vp, vp, vp]
+        L.nm_export_sizes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
+        L.nm_query.argtypes = [vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i32),
+                               ctypes.POINTER(i32), ctypes.POINTER(i32)]
+        L.nm_device_status.argtypes = [vp]
+        L.nm_destroy.argtypes = [vp]
+        L.nm_destroy.restype = None
+        L.nm_last_error.restype = ctypes.c_char_p
+        L.nm_version.restype = ctypes.c_char_p
+        for name in ("nm_compress", "nm_recompress", "nm_spmm", "nm_test_spmm_skip_stage", "nm_decompress", "nm_export",
+                     "nm_export_sizes", "nm_query", "nm_device_status"):
+            getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != NM_OK:
+        raise NMError(status, lib().nm_last_error().decode(errors="replace"))
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+class NMHandle:
+    """One compressed weight (owns the library handle and its device memory)."""
+
+    def __init__(self, raw: int, n_out: int, k: int, N: int, M: int, dt: int):
+        self._raw = ctypes.c_void_p(raw)
+        self.n_out, self.k, self.N, self.M, self.dt = n_out, k, N, M, dt
+
+    @property
+    def raw(self) -> ctypes.c_void_p:
+        if not self._raw:
+            raise RuntimeError("handle already destroyed")
+        return self._raw
+
+    @property
+    def dtype(self) -> torch.dtype:
+        return _ELEM[self.dt]
+
+    def destroy(self) -> None:
+        if self._raw and _lib is not None:
+            _lib.nm_destroy(self._raw)
+        self._raw = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def nm_compress(W: torch.Tensor, N: int, M: int, stream=None) -> NMHandle:
+    """Prune W [n_out, k] (int8 / fp16 / bf16, on the GPU) to N:M and pack it."""
+    if not W.is_cuda:
+        raise ValueError("W must be a CUDA tensor")
+    if W.dtype not in _TORCH_DT:
+        raise ValueError(f"unsupported dtype {W.dtype}")
+    W = W.contiguous()
+    n_out, k = W.shape
+    out = ctypes.c_void_p()
+    _check(lib().nm_compress(_ptr(W), n_out, k, _TORCH_DT[W.dtype], N, M, _stream(stream), ctypes.byref(out)))
+    return NMHandle(out.value, n_out, k, N, M, _TORCH_DT[W.dtype])
+
+
+def nm_recompress(h: NMHandle, W: torch.Tensor, stream=None) -> NMHandle:
+    """Re-prune and re-pack a new weight of the same shape/dtype into ``h`` (no allocation)."""
+    if not W.is_cuda or W.dtype != h.dtype or tuple(W.shape) != (h.n_out, h.k) or not W.is_contiguous():
+        raise ValueError("W must be a contiguous CUDA tensor of the handle's shape and dtype")
+    _check(lib().nm_recompress(h.raw, _ptr(W), _stream(stream)))
+    return h
+
+
+def out_dtype(h: NMHandle, scaled: bool) -> torch.dtype:
+    if h.dt == NM_INT8:
+        return torch.float32 if scaled else torch.int32
+    return _ELEM[h.dt]
+
+
+def nm_spmm(h: NMHandle, X: torch.Tensor, Y: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """Y = X @ Wm^T for the compressed weight of ``h`` (see include/nmspmm.h)."""
+    if X.dtype != h.dtype or not X.is_cuda or not X.is_contiguous() or X.dim() != 2 or X.shape[1] != h.k:
+        raise ValueError("X must be a contiguous CUDA [T, k] tensor of the handle's dtype")
+    T = X.shape[0]
+    want = out_dtype(h, scale is not None)
+    if Y is None:
+        Y = torch.empty((T, h.n_out), dtype=want, device=X.device)
+    elif Y.dtype != want or tuple(Y.shape) != (T, h.n_out) or not Y.is_contiguous():
+        raise ValueError(f"Y must be a contiguous [{T}, {h.n_out}] {want} tensor")
+    if scale is not None and (scale.dtype != torch.float32 or scale.numel() != h.n_out or not scale.is_cuda):
+        raise ValueError("scale must be a CUDA float32 tensor of n_out elements")
+    _check(lib().nm_spmm(h.raw, _ptr(X), T, _ptr(Y), _ptr(scale), _stream(stream)))
+    return Y
+
+
+def nm_test_spmm_skip_stage(h: NMHandle, X: torch.Tensor, Y: torch.Tensor, scale: torch.Tensor | None,
+                            skip_stage: int, timeout_ns: int, stream=None) -> int:
+    """Test hook: run the SpMM with one producer stage left unfilled; returns the launch status."""
+    return lib().nm_test_spmm_skip_stage(h.raw, _ptr(X), X.shape[0], _ptr(Y), _ptr(scale), _stream(stream),
+                                         skip_stage, timeout_ns)
+
+
+def nm_decompress(h: NMHandle, stream=None) -> torch.Tensor:
+    """Masked dense W decoded from the packed operand image the SpMM reads."""
+    out = torch.empty((h.n_out, h.k), dtype=h.dtype, device="cuda")
+    _check(lib().nm_decompress(h.raw, _ptr(out), _stream(stream)))
+    return out
+
+
+def nm_export_sizes(h: NMHandle) -> tuple[int, int]:
+    vb, ib = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().nm_export_sizes(h.raw, ctypes.byref(vb), ctypes.byref(ib)))
+    return vb.value, ib.value
+
+
+def nm_export(h: NMHandle):
+    """Canonical format on the host: (values [n_out, k/M, N], idx [n_out, pitch] uint8) as torch CPU tensors."""
+    vb, ib = nm_export_sizes(h)
+    values = torch.empty((h.n_out, h.k // h.M, h.N), dtype=h.dtype)
+    idx = torch.empty((h.n_out, ib // h.n_out), dtype=torch.uint8)
+    assert values.numel() * values.element_size() == vb
+    _check(lib().nm_export(h.raw, _ptr(values), _ptr(idx)))
+    return values, idx
+
+
+def nm_query(h: NMHandle) -> dict:
+    n, k, N, M, dt = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib().nm_query(h.raw, ctypes.byref(n), ctypes.byref(k), ctypes.byref(N), ctypes.byref(M),
+                          ctypes.byref(dt)))
+    return {"n_out": n.value, "k": k.value, "N": N.value, "M": M.value, "dtype": dt.value}
+
+
+def nm_device_status(h: NMHandle) -> int:
+    """NM_OK, or NM_ERR_TIMEOUT if a kernel gave up a bounded wait (clears the word)."""
+    return lib().nm_device_status(h.raw)
+
+
+def nm_last_error() -> str:
+    return lib().nm_last_error().decode(errors="replace")
+
+
+def nm_version() -> str:
+    return lib().nm_version().decode()

@@ -1,0 +1,374 @@
+// nm_api.cu -- the C ABI of libnmspmm (declared in include/nmspmm.h):
+// argument validation, handle lifetime, the per-shape launch plan (adaptive
+// parallelism, "Realizable N:M Sparse Transformer Inference via Search-Kernel
+// Co-Design", section 4.1 mechanism 3), activation tensor maps and the split-K
+// workspace.  All arithmetic runs in the kernels of nm_pack.cu / nm_spmm.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "../../include/nmspmm.h"
+#include "nm_device.cuh"
+#include "nm_internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+nm_status fail(nm_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+nm_status fail(nm_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+nm_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(e == cudaErrorMemoryAllocation ? NM_ERR_OOM : NM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int num_sms(int dev) {
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  return (v && *v) ? atoi(v) : dflt;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Activation X [T][k] as a 2-D tensor: inner dim k, box = 128 bytes x bn rows,
+// 128-byte swizzle (the layout the MMA's K-major B descriptor expects);
+// out-of-range rows and columns read as zero.
+nm_status make_x_map(nm_handle* h, const void* X, int64_t T, int bn) {
+  if (h->tm_x == X && h->tm_T == T && h->tm_bn == bn) return NM_OK;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int es = nm::elem_bytes(h->dt);
+  CUtensorMapDataType ty = h->dt == nm::DT_I8    ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                           : h->dt == nm::DT_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[2] = {(cuuint64_t)h->k, (cuuint64_t)T};
+  cuuint64_t strides[1] = {(cuuint64_t)(h->k * es)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)bn};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&h->tm, ty, 2, const_cast<void*>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    h->tm_x = nullptr;
+    return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for T=%lld k=%lld", (int)r, (long long)T,
+                (long long)h->k);
+  }
+  h->tm_x = X;
+  h->tm_T = T;
+  h->tm_bn = bn;
+  return NM_OK;
+}
+
+// Adaptive parallelism: pick the token tile and split-K factor for this shape.
+// Token tile: minimise (waves of persistent CTAs) x (per-tile cost ~ bn + 32).
+// Split-K: only when even the smallest tile leaves most SMs idle; partials are
+// reduced by the last-arriving CTA, so the reduction costs one extra pass over
+// the tile per split, which is why splits stay bounded by the idle SMs.
+nm::Plan make_plan(const nm_handle* h, int64_t T, int sms) {
+  nm::Plan p;
+  const int forced_bn = env_int("NMSPMM_FORCE_BN", 0);
+  const int forced_split = env_int("NMSPMM_FORCE_SPLITK", 0);
+  const int bns[3] = {128, 64, 32};
+  double best = 1e300;
+  for (int bn : bns) {
+    if (forced_bn && bn != forced_bn) continue;
+    const int64_t tiles = (int64_t)h->n_ct * ((T + bn - 1) / bn);
+    const int64_t waves = (tiles + sms - 1) / sms;
+    const double cost = (double)waves * (bn + 32);
+    if (cost < best) {
+      best = cost;
+      p.bn = bn;
+    }
+  }
+  p.n_tt = (int)((T + p.bn - 1) / p.bn);
+  const int64_t tiles = (int64_t)h->n_ct * p.n_tt;
+  int splits = 1;
+  if (forced_split > 0) {
+    splits = forced_split;
+  } else if (tiles * 2 <= sms && h->n_kb >= 2) {
+    splits = (int)std::min<int64_t>(h->n_kb, sms / tiles);
+  }
+  splits = std::max(1, std::min(splits, h->n_kb));
+  p.kb_per_split = (h->n_kb + splits - 1) / splits;
+  p.splits = (h->n_kb + p.kb_per_split - 1) / p.kb_per_split;  // every split owns >= 1 k-block
+  p.units = (int)(tiles * p.splits);
+  p.grid = std::min(p.units, sms);
+  return p;
+}
+
+nm_status check_handle(const nm_handle* h) {
+  if (!h) return fail(NM_ERR_INVALID, "null handle");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device)
+    return fail(NM_ERR_INVALID, "handle belongs to device %d but the current device is %d", h->device, dev);
+  return NM_OK;
+}
+
+nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, const float* scale, void* stream,
+                    int inject_skip, unsigned long long timeout_ns) {
+  g_err.clear();
+  nm_status st = check_handle(hc);
+  if (st != NM_OK) return st;
+  nm_handle* h = const_cast<nm_handle*>(hc);  // only caches (tensor map, workspace) change
+  if (T < 0) return fail(NM_ERR_INVALID, "T must be >= 0 (got %lld)", (long long)T);
+  if (T == 0) return NM_OK;
+  if (!X || !Y) return fail(NM_ERR_INVALID, "null X or Y");
+  if (T > INT32_MAX) return fail(NM_ERR_UNSUPPORTED, "T above 2^31-1");
+  const int es = nm::elem_bytes(h->dt);
+  if (!aligned(X, 16) || !aligned(Y, 16)) return fail(NM_ERR_INVALID, "X and Y must be 16-byte aligned");
+  if ((h->k * es) % 16 != 0)
+    return fail(NM_ERR_UNSUPPORTED, "k * sizeof(dtype) must be a multiple of 16 bytes (k=%lld)", (long long)h->k);
+  if (scale && !aligned(scale, 4)) return fail(NM_ERR_INVALID, "scale must be 4-byte aligned");
+  const size_t ybytes = (size_t)T * h->n_out * ((h->dt == nm::DT_I8) ? 4 : 2);
+  const size_t xbytes = (size_t)T * h->k * es;
+  const uintptr_t xs = (uintptr_t)X, ys = (uintptr_t)Y;
+  if (xs < ys + ybytes && ys < xs + xbytes) return fail(NM_ERR_INVALID, "Y overlaps X");
+
+  const int sms = num_sms(h->device);
+  nm::Plan p = make_plan(h, T, sms);
+  st = make_x_map(h, X, T, p.bn);
+  if (st != NM_OK) return st;
+
+  nm::SpmmArgs a{};
+  a.bpack = h->d_bpack;
+  a.Y = Y;
+  a.scale = scale;
+  a.err = h->d_err;
+  a.T = (int)T;
+  a.n_out = (int)h->n_out;
+  a.n_kb = h->n_kb;
+  a.n_ct = h->n_ct;
+  a.n_tt = p.n_tt;
+  a.splits = p.splits;
+  a.kb_per_split = p.kb_per_split;
+  a.units = p.units;
+  a.timeout_ns = timeout_ns;
+  a.inject_skip = inject_skip;
+  if (p.splits > 1) {
+    const int tiles = h->n_ct * p.n_tt;
+    const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
+    if (need > h->ws_bytes || tiles > h->cnt_len) {
+      cudaError_t e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) return cuda_fail(e, "synchronise before growing the split-K workspace");
+      cudaFree(h->d_ws);
+      cudaFree(h->d_cnt);
+      h->d_ws = nullptr;
+      h->d_cnt = nullptr;
+      h->ws_bytes = 0;
+      h->cnt_len = 0;
+      const size_t ws = std::max(need, h->ws_bytes);
+      const int cl = std::max(tiles, 256);
+      if ((e = cudaMalloc(&h->d_ws, ws)) != cudaSuccess) return cuda_fail(e, "allocate split-K workspace");
+      if ((e = cudaMalloc(&h->d_cnt, (size_t)cl * sizeof(int))) != cudaSuccess)
+        return cuda_fail(e, "allocate split-K counters");
+      if ((e = cudaMemset(h->d_cnt, 0, (size_t)cl * sizeof(int))) != cudaSuccess)
+        return cuda_fail(e, "clear split-K counters");
+      h->ws_bytes = ws;
+      h->cnt_len = cl;
+    }
+    a.ws = h->d_ws;
+    a.cnt = h->d_cnt;
+  }
+  cudaError_t e = nm::launch_spmm(h, &h->tm, p, a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launch SpMM kernel");
+  return NM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nm_last_error(void) { return g_err.c_str(); }
+
+const char* nm_version(void) { return "nmspmm 0.1.0 (sm_100a)"; }
+
+nm_status nm_compress(const void* W_dev, int64_t n_out, int64_t k, nm_dtype dt, int N, int M, void* stream,
+                      nm_handle** out) {
+  g_err.clear();
+  if (!out) return fail(NM_ERR_INVALID, "null output handle pointer");
+  *out = nullptr;
+  if (!W_dev) return fail(NM_ERR_INVALID, "null W");
+  if ((int)dt < 0 || (int)dt > 2) return fail(NM_ERR_INVALID, "unknown dtype %d", (int)dt);
+  if (n_out <= 0 || k <= 0) return fail(NM_ERR_INVALID, "n_out and k must be positive");
+  if (n_out > (1 << 24) || k > (1 << 24)) return fail(NM_ERR_UNSUPPORTED, "n_out and k are limited to 2^24");
+  if (M <= 0 || N <= 0 || N > M) return fail(NM_ERR_INVALID, "bad N:M %d:%d", N, M);
+  const bool sp24 = (N == 1 && M == 4) || (N == 2 && M == 4) || (N == 2 && M == 8);
+  const bool dense = (N == 4 && M == 8) || (N == M && (M == 4 || M == 8));
+  if (!sp24 && !dense) return fail(NM_ERR_UNSUPPORTED, "N:M %d:%d is not supported", N, M);
+  if (k % M != 0) return fail(NM_ERR_INVALID, "k=%lld is not a multiple of M=%d", (long long)k, M);
+  const int es = nm::elem_bytes((int)dt);
+  if (!aligned(W_dev, (size_t)es)) return fail(NM_ERR_INVALID, "W is not element aligned");
+
+  nm_handle* h = new (std::nothrow) nm_handle();
+  if (!h) return fail(NM_ERR_OOM, "host allocation failed");
+  cudaGetDevice(&h->device);
+  h->n_out = n_out;
+  h->k = k;
+  h->N = N;
+  h->M = M;
+  h->dt = (int)dt;
+  h->img = sp24 ? nm::IMG_SP24 : nm::IMG_DENSE;
+  const int KB = nm::kblock_elems(h->dt);
+  h->n_kb = (int)((k + KB - 1) / KB);
+  h->n_ct = (int)((n_out + nm::kRows - 1) / nm::kRows);
+  h->chunk = (size_t)nm::chunk_bytes(h->dt, h->img);
+  h->values_bytes = (size_t)n_out * (size_t)(k / M) * N * es;
+  h->idx_pitch = ((k / M) * N + 1) / 2;
+  h->idx_bytes = (size_t)n_out * (size_t)h->idx_pitch;
+  h->bpack_bytes = (size_t)h->n_ct * h->n_kb * h->chunk;
+
+  cudaError_t e;
+  nm_status st = NM_OK;
+  if ((e = cudaMalloc(&h->d_values, h->values_bytes)) != cudaSuccess) st = cuda_fail(e, "allocate values");
+  else if ((e = cudaMalloc(&h->d_idx, h->idx_bytes)) != cudaSuccess) st = cuda_fail(e, "allocate idx");
+  else if ((e = cudaMalloc(&h->d_bpack, h->bpack_bytes)) != cudaSuccess) st = cuda_fail(e, "allocate packed image");
+  else if ((e = cudaMalloc(&h->d_err, sizeof(int))) != cudaSuccess) st = cuda_fail(e, "allocate error word");
+  else if ((e = cudaMemsetAsync(h->d_err, 0, sizeof(int), (cudaStream_t)stream)) != cudaSuccess)
+    st = cuda_fail(e, "clear error word");
+  else if ((e = nm::launch_compress(h, W_dev, (cudaStream_t)stream)) != cudaSuccess)
+    st = cuda_fail(e, "launch compress kernel");
+  if (st != NM_OK) {
+    const std::string msg = g_err;
+    nm_destroy(h);
+    g_err = msg;
+    return st;
+  }
+  *out = h;
+  return NM_OK;
+}
+
+nm_status nm_recompress(nm_handle* h, const void* W_dev, void* stream) {
+  g_err.clear();
+  nm_status st = check_handle(h);
+  if (st != NM_OK) return st;
+  if (!W_dev) return fail(NM_ERR_INVALID, "null W");
+  if (!aligned(W_dev, (size_t)nm::elem_bytes(h->dt))) return fail(NM_ERR_INVALID, "W is not element aligned");
+  cudaError_t e = nm::launch_compress(h, W_dev, (cudaStream_t)stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch compress kernel");
+}
+
+nm_status nm_spmm(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev, const float* scale_dev,
+                  void* stream) {
+  return spmm_impl(h, X_dev, T, Y_dev, scale_dev, stream, -1, 1000000000ull);
+}
+
+nm_status nm_test_spmm_skip_stage(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
+                                  const float* scale_dev, void* stream, int skip_stage, int64_t timeout_ns) {
+  if (timeout_ns <= 0 || timeout_ns > 2000000000ll) return fail(NM_ERR_INVALID, "timeout must be in (0, 2 s]");
+  return spmm_impl(h, X_dev, T, Y_dev, scale_dev, stream, skip_stage, (unsigned long long)timeout_ns);
+}
+
+nm_status nm_decompress(const nm_handle* h, void* W_dev_out, void* stream) {
+  g_err.clear();
+  nm_status st = check_handle(h);
+  if (st != NM_OK) return st;
+  if (!W_dev_out) return fail(NM_ERR_INVALID, "null output");
+  if (!aligned(W_dev_out, 16)) return fail(NM_ERR_INVALID, "output must be 16-byte aligned");
+  cudaError_t e = nm::launch_decompress(h, W_dev_out, (cudaStream_t)stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch decompress kernel");
+}
+
+nm_status nm_export_sizes(const nm_handle* h, size_t* values_bytes, size_t* idx_bytes) {
+  g_err.clear();
+  if (!h) return fail(NM_ERR_INVALID, "null handle");
+  if (values_bytes) *values_bytes = h->values_bytes;
+  if (idx_bytes) *idx_bytes = h->idx_bytes;
+  return NM_OK;
+}
+
+nm_status nm_export(const nm_handle* h, void* values_host, uint8_t* idx_host) {
+  g_err.clear();
+  nm_status st = check_handle(h);
+  if (st != NM_OK) return st;
+  if (!values_host || !idx_host) return fail(NM_ERR_INVALID, "null host buffer");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "synchronise before export");
+  if ((e = cudaMemcpy(values_host, h->d_values, h->values_bytes, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "copy values");
+  if ((e = cudaMemcpy(idx_host, h->d_idx, h->idx_bytes, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "copy idx");
+  return NM_OK;
+}
+
+nm_status nm_query(const nm_handle* h, int64_t* n_out, int64_t* k, int* N, int* M, nm_dtype* dt) {
+  g_err.clear();
+  if (!h) return fail(NM_ERR_INVALID, "null handle");
+  if (n_out) *n_out = h->n_out;
+  if (k) *k = h->k;
+  if (N) *N = h->N;
+  if (M) *M = h->M;
+  if (dt) *dt = (nm_dtype)h->dt;
+  return NM_OK;
+}
+
+nm_status nm_device_status(const nm_handle* h) {
+  g_err.clear();
+  nm_status st = check_handle(h);
+  if (st != NM_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "synchronise");
+  int word = 0;
+  if ((e = cudaMemcpy(&word, h->d_err, sizeof word, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "read error word");
+  if (word == 0) return NM_OK;
+  cudaMemset(h->d_err, 0, sizeof(int));
+  static const char* where[] = {"", "producer waiting for a free stage", "MMA waiting for a free accumulator",
+                                "MMA waiting for operands", "epilogue waiting for an accumulator"};
+  return fail(NM_ERR_TIMEOUT, "a kernel gave up a bounded wait (%s)", (word >= 1 && word <= 4) ? where[word] : "?");
+}
+
+void nm_destroy(nm_handle* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  cudaFree(h->d_values);
+  cudaFree(h->d_idx);
+  cudaFree(h->d_bpack);
+  cudaFree(h->d_err);
+  cudaFree(h->d_ws);
+  cudaFree(h->d_cnt);
+  delete h;
+}
+
+}  // extern "C"

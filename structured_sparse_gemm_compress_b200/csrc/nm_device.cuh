@@ -1,0 +1,254 @@
+// nm_device.cuh -- device-side building blocks of the sm_100a N:M sparse GEMM:
+// the packed weight image layout ("B_pack") and thin inline-PTX wrappers for
+// mbarriers, bulk/tensor copies and the 5th-generation tensor core (tcgen05).
+//
+// Packed image (paper "Realizable N:M Sparse Transformer Inference via
+// Search-Kernel Co-Design", section 4.2: values and their in-window positions
+// are packed together so no separate index load is needed).  The image is a
+// sequence of chunks, one per (128-row channel tile ct, k-block kb), chunk
+// (ct, kb) at byte (ct * n_kb + kb) * chunk_bytes.  A k-block covers KB dense k
+// positions: 256 for INT8, 128 for FP16/BF16, i.e. 256 bytes of X per token.
+//
+//   2:4-image chunk (patterns 1:4, 2:4, 2:8; two slots per group of four):
+//     [ A: 128 rows x 128 B ]  compressed values, row r = channel ct*128 + r,
+//                              stored as the tensor core's K-major 128-byte
+//                              swizzled operand (16-byte unit c of row r sits at
+//                              unit c ^ (r & 7)).
+//     [ E: metadata ]          two 2-bit positions per group of four dense k
+//                              (nibble = pos0 | pos1 << 2, pos0 < pos1), laid out
+//                              so one tcgen05.cp per 128 rows x 16 bytes puts it
+//                              where the sparse MMA reads it:
+//                INT8 (4096 B): half h of the block (dense k [128h, 128h+128))
+//                               at 2048*h; row r at 16*r; bit (k mod 128).
+//                FP16/BF16 (2048 B): row r = m0 + 8*m1 + 16*m2 and dense k =
+//                               k0 + 16*k1 + 32*k2 go to 16-byte line
+//                               m0 + 8*k1 + 16*m2, bit 32*k2 + 16*m1 + k0.
+//   dense-image chunk (pattern 4:8 and N == M): [ A: two 128 x 128 B swizzled
+//     atoms ] holding the masked dense tile (bytes [128a, 128a+128) of each
+//     row in atom a).
+// Rows beyond n_out and k beyond K are zero (metadata nibble 0).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace nm {
+
+enum : int { DT_I8 = 0, DT_F16 = 1, DT_BF16 = 2 };
+enum : int { IMG_SP24 = 0, IMG_DENSE = 1 };
+
+constexpr int kRows = 128;          // channel rows per tile (MMA M)
+constexpr int kAtomBytes = 16384;   // 128 rows x 128 B swizzled atom
+
+__host__ __device__ constexpr int kblock_elems(int dt) { return dt == DT_I8 ? 256 : 128; }
+__host__ __device__ constexpr int elem_bytes(int dt) { return dt == DT_I8 ? 1 : 2; }
+__host__ __device__ constexpr int meta_bytes(int dt) { return dt == DT_I8 ? 4096 : 2048; }
+__host__ __device__ constexpr int chunk_bytes(int dt, int img) {
+  return img == IMG_SP24 ? kAtomBytes + meta_bytes(dt) : 2 * kAtomBytes;
+}
+
+// Byte offset of (row r, byte c of the 128-byte row) inside a swizzled atom.
+__host__ __device__ inline uint32_t swz128(uint32_t r, uint32_t c) {
+  return r * 128u + ((((c >> 4) ^ r) & 7u) << 4) + (c & 15u);
+}
+
+// Byte offset inside the metadata block of the 16 bits that hold the four
+// nibbles of dense k [kk, kk+16) (kk a multiple of 16) for tile row r.
+__host__ __device__ inline uint32_t meta_off16(int dt, uint32_t r, uint32_t kk) {
+  if (dt == DT_I8) return (kk >> 7) * 2048u + r * 16u + ((kk & 127u) >> 3);
+  const uint32_t m0 = r & 7u, m1 = (r >> 3) & 1u, m2 = r >> 4;
+  const uint32_t k1 = (kk >> 4) & 1u, k2 = kk >> 5;
+  const uint32_t line = m0 + 8u * k1 + 16u * m2;
+  return line * 16u + 4u * k2 + 2u * m1;
+}
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of parity `parity` to complete, giving up after
+// `timeout_ns` or as soon as *abort is set.  Returns false when it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > timeout_ns) return false;
+    }
+  }
+}
+
+// One contiguous global -> shared copy completing on `bar` (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 2-D tiled tensor copy (no multicast) completing on `bar`; c0 is the inner coordinate.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                            int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// --- tcgen05 (tensor memory + 5th-generation MMA)
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand with 128-byte swizzle,
+// 8-row groups 1024 bytes apart (version 1 = sm_100 format).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;                 // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset: next 8-row group
+  d |= (uint64_t)1u << 46;                 // descriptor version
+  d |= (uint64_t)2u << 61;                 // layout: 128-byte swizzle
+  return d;
+}
+
+// Shared-memory descriptor of an unswizzled 128-row x 16-byte block (rows 16 B
+// apart, 8-row groups 128 B apart), the source of a 128x128b tcgen05.cp.
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128u >> 4) << 16;        // leading byte offset
+  d |= (uint64_t)(128u >> 4) << 32;        // stride byte offset
+  d |= (uint64_t)1u << 46;
+  return d;                                // layout 0: no swizzle
+}
+
+__device__ __forceinline__ void tc_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+template <int KIND>  // 0: kind::i8, 1: kind::f16
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  if constexpr (KIND == 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ void tc_mma_sp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
+                                          uint32_t idesc, uint32_t accumulate) {
+  if constexpr (KIND == 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
+// Arrive on `bar` once every tcgen05 operation issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives its lane's 32 columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+}  // namespace nm

@@ -1,0 +1,71 @@
+// nm_internal.h -- declarations shared by the host-side translation units of
+// libnmspmm (not part of the public ABI; see include/nmspmm.h for that).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+struct nm_handle {
+  int64_t n_out = 0, k = 0;
+  int N = 0, M = 0;
+  int dt = 0;            // nm::DT_*
+  int img = 0;           // nm::IMG_*
+  int n_kb = 0;          // k-blocks in the packed image
+  int n_ct = 0;          // 128-row channel tiles
+  size_t chunk = 0;      // bytes per (channel tile, k-block) chunk
+  int device = 0;
+
+  void* d_values = nullptr;   // canonical values [n_out][k/M][N]
+  uint8_t* d_idx = nullptr;   // canonical 4-bit positions [n_out][idx_pitch]
+  size_t values_bytes = 0, idx_bytes = 0;
+  int64_t idx_pitch = 0;
+  uint8_t* d_bpack = nullptr; // packed operand image
+  size_t bpack_bytes = 0;
+  int* d_err = nullptr;       // device error word (bounded-wait timeouts)
+
+  // split-K workspace (partials + per-tile arrival counters), grown on demand
+  void* d_ws = nullptr;
+  size_t ws_bytes = 0;
+  int* d_cnt = nullptr;
+  int cnt_len = 0;
+
+  // cached tensor map of the last activation seen
+  const void* tm_x = nullptr;
+  int64_t tm_T = -1;
+  int tm_bn = 0;
+  alignas(64) CUtensorMap tm;
+};
+
+namespace nm {
+
+// Launch plan chosen per problem (inference-aware adaptive parallelism).
+struct Plan {
+  int bn = 128;       // token tile (MMA N)
+  int splits = 1;     // split-K factor
+  int kb_per_split = 1;
+  int n_tt = 1;       // token tiles
+  int units = 1;      // (tile, split) work units
+  int grid = 1;       // persistent CTAs
+};
+
+struct SpmmArgs {
+  const uint8_t* bpack;
+  void* Y;
+  const float* scale;
+  void* ws;
+  int* cnt;
+  int* err;
+  int T, n_out, n_kb, n_ct, n_tt, splits, kb_per_split, units;
+  unsigned long long timeout_ns;
+  int inject_skip;    // test hook: producer omits the stage with this index (-1: never)
+};
+
+cudaError_t launch_compress(const nm_handle* h, const void* W, cudaStream_t s);
+cudaError_t launch_decompress(const nm_handle* h, void* Wout, cudaStream_t s);
+cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a,
+                        cudaStream_t s);
+size_t spmm_smem_bytes(int dt, int img, int bn);
+
+}  // namespace nm

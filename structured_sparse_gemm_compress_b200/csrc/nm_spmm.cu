@@ -1,0 +1,426 @@
+// nm_spmm.cu -- the micro-dense N:M SpMM kernel for sm_100a.
+//
+// Implements the execution side of "Realizable N:M Sparse Transformer Inference
+// via Search-Kernel Co-Design":
+//   * section 4.2, micro-dense execution: only the kept values of every window
+//     reach the tensor core, as regular dense operand tiles; the positions ride
+//     along in the same packed chunk and feed the sparse MMA's metadata, so
+//     the runtime compute is MMA only;
+//   * section 4.1, mechanism (3), adaptive parallelism: the host picks the
+//     token tile and a split-K factor per shape (nm_api.cu); split partials are
+//     reduced by the last-arriving CTA of a tile, so no CTA ever waits on
+//     another.
+//
+// Y^T tile [128 channels x BN tokens] = sum over k-blocks of
+//     MMA( W_tile [128 x k-block] (sparse 2:4 image or dense),
+//          X_tile [BN x k-block] (K-major) )
+// accumulated in tensor memory, so TMEM lane = output channel and TMEM column
+// = token; the epilogue therefore stores 32 consecutive channels of one token
+// per warp instruction (128 B, coalesced) without a transpose.
+//
+// CTA = 6 warps, one persistent CTA per SM:
+//   warp 0      producer: one bulk copy of the packed weight chunk (values +
+//               positions) and two 2-D tensor copies of X per stage;
+//   warp 1      TMEM owner and MMA issuer (one thread): copies the positions
+//               into TMEM (tcgen05.cp) and issues tcgen05.mma(.sp);
+//   warps 2..5  epilogue: tcgen05.ld, optional per-channel scale, stores.
+// Two TMEM accumulators let the epilogue of one tile overlap the mainloop of
+// the next.  Every wait is bounded; on a timeout the kernel records an error
+// word, drains its own copies and MMAs, frees TMEM and returns.
+#include "nm_device.cuh"
+#include "nm_internal.h"
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace nm {
+
+enum : int { OUT_I32 = 0, OUT_F32 = 1, OUT_F16 = 2, OUT_BF16 = 3 };
+
+constexpr int kThreads = 192;
+constexpr int kSmemBudget = 227 * 1024 - 1024;  // dynamic shared memory after 1 KB alignment slack
+
+template <int DT, int IMG, int BN>
+struct Cfg {
+  static constexpr bool SP = IMG == IMG_SP24;
+  static constexpr int KB = kblock_elems(DT);
+  static constexpr int CHUNK = chunk_bytes(DT, IMG);
+  static constexpr int B_BOX = BN * 128;            // one 128-byte-wide box of X rows
+  static constexpr int STAGE = CHUNK + 2 * B_BOX;   // multiple of 1024
+  static constexpr int STAGES = (kSmemBudget / STAGE) > 8 ? 8 : (kSmemBudget / STAGE);
+  static constexpr int MMAS = SP ? 4 : 8;           // MMAs per stage (each 32 B of A per row)
+  static constexpr int E_COLS = SP ? (DT == DT_I8 ? 8 : 4) : 0;
+  static constexpr int E_COL0 = 2 * BN;             // metadata slots after the two accumulators
+  static constexpr int COLS_NEEDED = 2 * BN + 2 * E_COLS;
+  static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 : COLS_NEEDED <= 128 ? 128
+                                   : COLS_NEEDED <= 256 ? 256 : 512;
+  static constexpr int SMEM = STAGES * STAGE + 1024;
+  static_assert(STAGE % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(STAGES >= 2, "need at least two stages");
+  static_assert(COLS_NEEDED <= 512, "tensor memory overflow");
+};
+
+// Instruction descriptor: A K-major (sparse or dense), B K-major, M = 128.
+template <int DT, bool SP, int BN>
+__host__ __device__ constexpr uint32_t make_idesc() {
+  uint32_t d = 0;
+  if (SP) d |= 1u << 2;                    // sparse A
+  if (DT == DT_I8) {
+    d |= 2u << 4;                          // D: s32
+    d |= 1u << 7;                          // A: signed 8-bit
+    d |= 1u << 10;                         // B: signed 8-bit
+  } else {
+    d |= 1u << 4;                          // D: f32
+    const uint32_t f = DT == DT_BF16 ? 1u : 0u;
+    d |= f << 7;                           // A: f16 / bf16
+    d |= f << 10;                          // B
+  }
+  d |= (uint32_t)(BN >> 3) << 17;          // N
+  d |= (uint32_t)(128 >> 4) << 24;         // M
+  return d;
+}
+
+struct Unit {
+  int ct, tt, z, tile, kb0, kb1;
+};
+__device__ __forceinline__ Unit decode_unit(int u, const SpmmArgs& a) {
+  Unit w;
+  w.tile = u / a.splits;
+  w.z = u - w.tile * a.splits;
+  w.ct = w.tile % a.n_ct;
+  w.tt = w.tile / a.n_ct;
+  w.kb0 = w.z * a.kb_per_split;
+  w.kb1 = min(a.n_kb, w.kb0 + a.kb_per_split);
+  return w;
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_out(void* Y, size_t i, uint32_t acc, float s, bool has_scale) {
+  if constexpr (OUT == OUT_I32) {
+    reinterpret_cast<int32_t*>(Y)[i] = (int32_t)acc;
+  } else if constexpr (OUT == OUT_F32) {
+    reinterpret_cast<float*>(Y)[i] = __fmul_rn(__int2float_rn((int32_t)acc), s);
+  } else {
+    float f = __uint_as_float(acc);
+    if (has_scale) f = __fmul_rn(f, s);
+    if constexpr (OUT == OUT_F16)
+      reinterpret_cast<__half*>(Y)[i] = __float2half_rn(f);
+    else
+      reinterpret_cast<__nv_bfloat16*>(Y)[i] = __float2bfloat16_rn(f);
+  }
+}
+
+// Sum of split partials (int32 for INT8, fp32 otherwise), in split order.
+template <int DT>
+__device__ __forceinline__ uint32_t add_acc(uint32_t x, uint32_t y) {
+  if constexpr (DT == DT_I8)
+    return (uint32_t)((int32_t)x + (int32_t)y);
+  else
+    return __float_as_uint(__uint_as_float(x) + __uint_as_float(y));
+}
+
+template <int DT, int IMG, int BN, int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
+  using C = Cfg<DT, IMG, BN>;
+  constexpr bool SP = C::SP;
+  constexpr int KIND = DT == DT_I8 ? 0 : 1;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t accf_bar[2];
+  __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+  __shared__ int last_sh;
+  __shared__ volatile int ep_ok_sh[2];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accf_bar[i], 1);
+      mbar_init(&acce_bar[i], 4);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&tmX);
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint64_t tmo = a.timeout_ns;
+
+  auto give_up = [&](int code) {
+    abort_sh = 1;
+    if (a.err) atomicExch(a.err, code);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0, seq = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;  // per stage: last use carried copies / its parity
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
+        const Unit w = decode_unit(u, a);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++seq) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
+            give_up(1);
+            ok = false;
+            break;
+          }
+          if (seq != a.inject_skip) {
+            uint8_t* st = smem + (size_t)stage * C::STAGE;
+            mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)C::STAGE);
+            bulk_load(st, a.bpack + ((size_t)w.ct * a.n_kb + kb) * C::CHUNK, (uint32_t)C::CHUNK,
+                      &full_bar[stage]);
+            tma_load_2d(st + C::CHUNK, &tmX, &full_bar[stage], kb * C::KB, w.tt * BN);
+            tma_load_2d(st + C::CHUNK + C::B_BOX, &tmX, &full_bar[stage], kb * C::KB + C::KB / 2, w.tt * BN);
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          } else {
+            armed &= ~(1u << stage);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: every copy this thread issued has landed before the CTA exits.
+      // Earlier uses of a stage were consumed before it was re-armed, so only
+      // the last armed use of each stage can still be in flight.
+      for (int i = 0; i < C::STAGES; ++i)
+        if ((armed >> i) & 1u) mbar_wait(&full_bar[i], (armed_par >> i) & 1u, &abort_sh, tmo);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc<DT, SP, BN>();
+      int stage = 0, acc = 0, eslot = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
+        const Unit w = decode_unit(u, a);
+        if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &abort_sh, tmo)) {
+          give_up(2);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_sh, tmo)) {
+            give_up(3);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + (size_t)stage * C::STAGE);
+          const uint32_t b_addr = a_addr + C::CHUNK;
+          uint32_t e_tmem = 0;
+          if constexpr (SP) {
+            e_tmem = tmem + (uint32_t)(C::E_COL0 + eslot * C::E_COLS);
+            const uint32_t e_addr = a_addr + kAtomBytes;
+            tc_cp_128x128b(e_tmem, sdesc_rows16(e_addr));
+            if constexpr (DT == DT_I8) tc_cp_128x128b(e_tmem + 4, sdesc_rows16(e_addr + 2048));
+          }
+#pragma unroll
+          for (int j = 0; j < C::MMAS; ++j) {
+            const uint32_t accum = (kb > w.kb0 || j > 0) ? 1u : 0u;
+            if constexpr (SP) {
+              const uint64_t ad = sdesc_sw128(a_addr + 32u * j);
+              const uint64_t bd = sdesc_sw128(b_addr + (uint32_t)((j >> 1) * C::B_BOX) + 64u * (j & 1));
+              uint32_t e_addr, id2;
+              if constexpr (DT == DT_I8) {
+                e_addr = e_tmem + 2u * j;
+                id2 = 0;
+              } else {
+                e_addr = e_tmem + (uint32_t)(j & ~1);
+                id2 = (uint32_t)(j & 1);
+              }
+              tc_mma_sp<KIND>(d_tmem, ad, bd, e_addr, idesc | id2, accum);
+            } else {
+              const uint64_t ad = sdesc_sw128(a_addr + (uint32_t)((j >> 2) * kAtomBytes) + 32u * (j & 3));
+              const uint64_t bd = sdesc_sw128(b_addr + (uint32_t)((j >> 2) * C::B_BOX) + 32u * (j & 3));
+              tc_mma<KIND>(d_tmem, ad, bd, idesc, accum);
+            }
+          }
+          tc_commit(&empty_bar[stage]);  // frees the smem stage once these MMAs have read it
+          eslot ^= 1;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&accf_bar[acc]);  // accumulator ready for the epilogue
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // Drain: all tcgen05 work issued by this thread completes before TMEM is freed.
+      tc_commit(&drain_bar);
+      mbar_wait(&drain_bar, 0, &abort_sh, tmo);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int lg = warp & 3;  // TMEM lane quarter this warp may access
+    const int ep_tid = threadIdx.x - 64;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    // One thread waits (bounded) and broadcasts the outcome, so all 128
+    // epilogue threads take the same branch and always meet at the named
+    // barriers; the flag alternates between two slots so a fast thread's next
+    // write cannot overtake a slow thread's read.
+    int iter = 0;
+    for (int u = blockIdx.x; u < a.units; u += gridDim.x, ++iter) {
+      const Unit w = decode_unit(u, a);
+      if (ep_tid == 0) {
+        const bool got = mbar_wait(&accf_bar[acc], acc_phase, &abort_sh, tmo);
+        if (!got) give_up(4);
+        ep_ok_sh[iter & 1] = got ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (!ep_ok_sh[iter & 1]) break;
+      tc_fence_after();
+      const int ch = w.ct * kRows + lg * 32 + lane;
+      const bool ch_ok = ch < a.n_out;
+      const bool has_scale = a.scale != nullptr;
+      const float s = (has_scale && ch_ok) ? __ldg(a.scale + ch) : 1.0f;
+      const int t0 = w.tt * BN;
+      const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(acc * BN);
+      if (a.splits == 1) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + 32u * c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = t0 + 32 * c + j;
+            if (ch_ok && t < a.T) store_out<OUT>(a.Y, (size_t)t * a.n_out + ch, r[j], s, has_scale);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce_bar[acc]);
+      } else {
+        // split-K: publish this split's partial tile, the last arriving split reduces
+        uint32_t* part = reinterpret_cast<uint32_t*>(a.ws);
+        const size_t tile_elems = (size_t)BN * kRows;
+        uint32_t* mine = part + ((size_t)w.tile * a.splits + w.z) * tile_elems;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + 32u * c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) __stcg(mine + (size_t)(32 * c + j) * kRows + lg * 32 + lane, r[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce_bar[acc]);
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (ep_tid == 0) last_sh = (atomicAdd(a.cnt + w.tile, 1) == a.splits - 1);
+        named_bar_sync(1, 128);
+        if (last_sh) {
+          __threadfence();
+          const uint32_t* tile_base = part + (size_t)w.tile * a.splits * tile_elems;
+#pragma unroll 1
+          for (int col = 0; col < BN; ++col) {
+            const int t = t0 + col;
+            if (t >= a.T) break;
+            const size_t off = (size_t)col * kRows + lg * 32 + lane;
+            uint32_t sum = __ldcg(tile_base + off);
+            for (int z = 1; z < a.splits; ++z) sum = add_acc<DT>(sum, __ldcg(tile_base + z * tile_elems + off));
+            if (ch_ok) store_out<OUT>(a.Y, (size_t)t * a.n_out + ch, sum, s, has_scale);
+          }
+          if (ep_tid == 0) a.cnt[w.tile] = 0;  // re-arm for the next launch
+        }
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host launch
+
+template <int DT, int IMG, int BN, int OUT>
+static cudaError_t launch_t(const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  using C = Cfg<DT, IMG, BN>;
+  auto kern = spmm_kernel<DT, IMG, BN, OUT>;
+  static bool attr_set = false;  // per instantiation; set once per process (single device use)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<p.grid, kThreads, C::SMEM, s>>>(*tmX, a);
+  return cudaGetLastError();
+}
+
+template <int DT, int IMG, int OUT>
+static cudaError_t launch_bn(const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  switch (p.bn) {
+    case 32: return launch_t<DT, IMG, 32, OUT>(tmX, p, a, s);
+    case 64: return launch_t<DT, IMG, 64, OUT>(tmX, p, a, s);
+    case 128: return launch_t<DT, IMG, 128, OUT>(tmX, p, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int DT, int OUT>
+static cudaError_t launch_img(int img, const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  return img == IMG_SP24 ? launch_bn<DT, IMG_SP24, OUT>(tmX, p, a, s) : launch_bn<DT, IMG_DENSE, OUT>(tmX, p, a, s);
+}
+
+cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a,
+                        cudaStream_t s) {
+  switch (h->dt) {
+    case DT_I8:
+      return a.scale ? launch_img<DT_I8, OUT_F32>(h->img, tmX, p, a, s)
+                     : launch_img<DT_I8, OUT_I32>(h->img, tmX, p, a, s);
+    case DT_F16: return launch_img<DT_F16, OUT_F16>(h->img, tmX, p, a, s);
+    default: return launch_img<DT_BF16, OUT_BF16>(h->img, tmX, p, a, s);
+  }
+}
+
+size_t spmm_smem_bytes(int dt, int img, int bn) {
+  auto pick = [&](auto c) { return (size_t)decltype(c)::SMEM; };
+  if (dt == DT_I8) {
+    if (img == IMG_SP24) return bn == 32 ? pick(Cfg<DT_I8, IMG_SP24, 32>{}) : bn == 64 ? pick(Cfg<DT_I8, IMG_SP24, 64>{}) : pick(Cfg<DT_I8, IMG_SP24, 128>{});
+    return bn == 32 ? pick(Cfg<DT_I8, IMG_DENSE, 32>{}) : bn == 64 ? pick(Cfg<DT_I8, IMG_DENSE, 64>{}) : pick(Cfg<DT_I8, IMG_DENSE, 128>{});
+  }
+  if (img == IMG_SP24) return bn == 32 ? pick(Cfg<DT_F16, IMG_SP24, 32>{}) : bn == 64 ? pick(Cfg<DT_F16, IMG_SP24, 64>{}) : pick(Cfg<DT_F16, IMG_SP24, 128>{});
+  return bn == 32 ? pick(Cfg<DT_F16, IMG_DENSE, 32>{}) : bn == 64 ? pick(Cfg<DT_F16, IMG_DENSE, 64>{}) : pick(Cfg<DT_F16, IMG_DENSE, 128>{});
+}
+
+}  // namespace nm

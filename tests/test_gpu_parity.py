@@ -1,0 +1,263 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+* compressed format (values + 4-bit positions): bit-exact;
+* masked weight decoded from the packed operand image: bit-exact;
+* INT8 SpMM (int32, and fp32 with per-channel scale): bit-exact;
+* FP16 SpMM: max |err| <= 2e-3 * max|Y_ref| and relative Frobenius error
+  <= 1e-3 against the fp64 oracle;
+* BF16 SpMM: max |err| <= 4e-3 * max|Y_ref|, relative Frobenius <= 2.5e-3
+  (bf16 keeps 8 significant bits: rounding the output once costs up to
+  2^-9 = 1.95e-3 relative per element, plus fp32 accumulation error).
+Sizes span several 128-channel and token tiles with ragged tails.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import structured_sparse_gemm_compress_b200 as nm
+from structured_sparse_gemm_compress_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+PATTERNS = [(1, 4), (2, 4), (2, 8), (4, 8), (4, 4), (8, 8)]
+TOL = {"fp16": (2e-3, 1e-3), "bf16": (4e-3, 2.5e-3)}
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_4x8.json")
+
+
+def _np(t: torch.Tensor, dtype: str) -> np.ndarray:
+    t = t.detach().cpu().contiguous()
+    if dtype == "bf16":
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def _weights(dtype, n_out, K, seed):
+    if dtype == "int8":
+        return inputs.int8_uniform((n_out, K), -127, 127, seed)
+    return inputs.float_normal((n_out, K), 0.02, seed, dtype)
+
+
+def _acts(dtype, T, K, seed):
+    if dtype == "int8":
+        return inputs.int8_uniform((T, K), -128, 127, seed)
+    return inputs.float_normal((T, K), 1.0, seed, dtype)
+
+
+def _assert_float_close(Y_gpu: torch.Tensor, Y_ref: np.ndarray, dtype: str):
+    got = Y_gpu.double().cpu().numpy()
+    err = np.abs(got - Y_ref)
+    mx = np.abs(Y_ref).max()
+    amax, frob = TOL[dtype]
+    assert err.max() <= amax * mx, (err.max(), mx)
+    assert np.linalg.norm(got - Y_ref) <= frob * np.linalg.norm(Y_ref)
+
+
+@pytest.fixture(autouse=True)
+def _no_forced_plan(monkeypatch):
+    monkeypatch.delenv("NMSPMM_FORCE_BN", raising=False)
+    monkeypatch.delenv("NMSPMM_FORCE_SPLITK", raising=False)
+
+
+# --------------------------------------------------------------------------- compress / decompress
+
+
+@pytest.mark.parametrize("dtype", ["int8", "fp16", "bf16"])
+@pytest.mark.parametrize("N,M", PATTERNS)
+@pytest.mark.parametrize("n_out,K", [(200, 784), (37, 40), (128, 256)])
+def test_compress_format_and_image_bit_exact(dtype, N, M, n_out, K):
+    W = _weights(dtype, n_out, K, seed=100 + n_out + K)
+    if dtype == "int8":  # plenty of exact ties and zeros
+        W = (W // 40).to(torch.int8)
+    h = nm.nm_compress(W.cuda(), N, M)
+    values, idx = nm.nm_export(h)
+    ref_v, ref_i = oracle.compress(_np(W, dtype), N, M, dtype)
+    assert np.array_equal(_np(values, dtype), ref_v)
+    assert np.array_equal(idx.numpy(), ref_i)
+    Wm = nm.nm_decompress(h)
+    torch.cuda.synchronize()
+    ref_Wm = oracle.decompress(ref_v, ref_i, n_out, K, N, M, dtype)
+    assert np.array_equal(_np(Wm, dtype), ref_Wm)
+
+
+def test_hand_examples_on_gpu():
+    g = json.load(open(GOLDEN))
+    W = torch.zeros((4, 16), dtype=torch.int8)
+    X = torch.zeros((2, 16), dtype=torch.int8)
+    W[:, :8] = torch.tensor(g["W"], dtype=torch.int8)   # zero groups appended: Y is unchanged
+    X[:, :8] = torch.tensor(g["X"], dtype=torch.int8)
+    for nm_str, case in g["cases"].items():
+        N, M = map(int, nm_str.split(":"))
+        h = nm.nm_compress(W.cuda(), N, M)
+        Y = nm.nm_spmm(h, X.cuda())
+        assert Y.cpu().tolist() == case["Y"], nm_str
+
+
+# --------------------------------------------------------------------------- SpMM parity
+
+
+@pytest.mark.parametrize("N,M", PATTERNS)
+@pytest.mark.parametrize("scaled", [False, True])
+@pytest.mark.parametrize("T,n_out,K", [(300, 200, 784), (1, 128, 256), (197, 96, 96), (64, 384, 3072)])
+def test_spmm_int8_bit_exact(N, M, scaled, T, n_out, K):
+    W = _weights("int8", n_out, K, seed=7 + K)
+    X = _acts("int8", T, K, seed=8 + T)
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=9) if scaled else None
+    h = nm.nm_compress(W.cuda(), N, M)
+    Y = nm.nm_spmm(h, X.cuda(), scale=None if s is None else s.cuda())
+    ref = oracle.spmm(X.numpy(), W.numpy(), N, M, scale=None if s is None else s.numpy())
+    got = Y.cpu().numpy()
+    assert got.dtype == ref.dtype
+    if scaled:
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    else:
+        assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("N,M", PATTERNS)
+@pytest.mark.parametrize("T,n_out,K", [(300, 200, 392), (5, 256, 1024), (131, 64, 4096)])
+def test_spmm_float_within_tolerance(dtype, N, M, T, n_out, K):
+    W = _weights(dtype, n_out, K, seed=17 + K)
+    X = _acts(dtype, T, K, seed=18 + T)
+    h = nm.nm_compress(W.cuda(), N, M)
+    Y = nm.nm_spmm(h, X.cuda())
+    ref = oracle.spmm(_np(X, dtype), _np(W, dtype), N, M, dtype=dtype)
+    _assert_float_close(Y, ref, dtype)
+
+
+def test_spmm_fp16_scaled():
+    W = _weights("fp16", 192, 512, seed=31)
+    X = _acts("fp16", 100, 512, seed=32)
+    s = inputs.scale_uniform(192, 0.5, 2.0, seed=33)
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
+    ref = oracle.spmm(_np(X, "fp16"), _np(W, "fp16"), 2, 4, scale=s.numpy(), dtype="fp16")
+    _assert_float_close(Y, ref, "fp16")
+
+
+@pytest.mark.parametrize("bn", ["32", "64", "128"])
+@pytest.mark.parametrize("split", ["1", "2", "3", "5"])
+def test_forced_tiles_and_splits_are_bit_identical(monkeypatch, bn, split):
+    """Adaptive parallelism must not change INT8 results at all."""
+    W = _weights("int8", 200, 1280, seed=41)
+    X = _acts("int8", 150, 1280, seed=42)
+    s = inputs.scale_uniform(200, 0.001, 0.01, seed=43)
+    ref = oracle.spmm(X.numpy(), W.numpy(), 2, 4, scale=s.numpy())
+    monkeypatch.setenv("NMSPMM_FORCE_BN", bn)
+    monkeypatch.setenv("NMSPMM_FORCE_SPLITK", split)
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    for _ in range(2):  # the second call reuses the re-armed split-K counters
+        Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
+        assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("split", ["1", "4"])
+def test_forced_split_fp16_within_tolerance(monkeypatch, split):
+    W = _weights("fp16", 256, 2048, seed=51)
+    X = _acts("fp16", 40, 2048, seed=52)
+    monkeypatch.setenv("NMSPMM_FORCE_SPLITK", split)
+    h = nm.nm_compress(W.cuda(), 2, 8)
+    Y = nm.nm_spmm(h, X.cuda())
+    _assert_float_close(Y, oracle.spmm(_np(X, "fp16"), _np(W, "fp16"), 2, 8, dtype="fp16"), "fp16")
+
+
+# --------------------------------------------------------------------------- full-size workloads (sampled)
+
+
+def _sampled_rows(T, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(T, size=min(count, T), replace=False).tolist())
+    rows.update({0, T - 1})
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("layer", inputs.single_layer(), ids=lambda l: l.name)
+def test_single_layer_full(layer):
+    W, X = layer.weight(), layer.activation()
+    h = nm.nm_compress(W.cuda(), layer.N, layer.M)
+    Y = nm.nm_spmm(h, X.cuda())
+    assert np.array_equal(Y.cpu().numpy(), oracle.spmm(X.numpy(), W.numpy(), layer.N, layer.M))
+
+
+@pytest.mark.parametrize("layer", inputs.vit_b_int8(), ids=lambda l: f"{l.name}-{l.nm}")
+def test_vit_b_int8_sampled_rows(layer):
+    W, X, s = layer.weight(), layer.activation(), layer.scale()
+    h = nm.nm_compress(W.cuda(), layer.N, layer.M)
+    Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
+    rows = _sampled_rows(layer.T, 48, layer.seed)
+    ref = oracle.spmm(X.numpy()[rows], W.numpy(), layer.N, layer.M, scale=s.numpy())
+    assert np.array_equal(Y.cpu().numpy()[rows].view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("layer", inputs.vit_l_fp16(), ids=lambda l: f"{l.name}-{l.nm}")
+def test_vit_l_fp16_sampled_rows(layer):
+    W, X = layer.weight(), layer.activation()
+    h = nm.nm_compress(W.cuda(), layer.N, layer.M)
+    Y = nm.nm_spmm(h, X.cuda())
+    rows = _sampled_rows(layer.T, 32, layer.seed)
+    ref = oracle.spmm(_np(X, "fp16")[rows], _np(W, "fp16"), layer.N, layer.M, dtype="fp16")
+    _assert_float_close(Y[rows.tolist()], ref, "fp16")
+
+
+@pytest.mark.parametrize("layer", inputs.swin_t_int8(), ids=lambda l: f"{l.name}-{l.nm}")
+def test_swin_t_int8_sampled_rows(layer):
+    W, X, s = layer.weight(), layer.activation(), layer.scale()
+    h = nm.nm_compress(W.cuda(), layer.N, layer.M)
+    Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
+    rows = _sampled_rows(layer.T, 48, layer.seed)
+    ref = oracle.spmm(X.numpy()[rows], W.numpy(), layer.N, layer.M, scale=s.numpy())
+    assert np.array_equal(Y.cpu().numpy()[rows].view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("T", [197, 50432])
+def test_vit_b_mixed_sequence(T):
+    """All 48 layers back to back in one stream; every layer checked (sampled rows at large T)."""
+    layers = inputs.vit_b_mixed(T)
+    outs = []
+    for l in layers:
+        W, X, s = l.weight(), l.activation(), l.scale()
+        h = nm.nm_compress(W.cuda(), l.N, l.M)
+        outs.append((l, X, W, s, h, nm.nm_spmm(h, X.cuda(), scale=s.cuda())))
+    torch.cuda.synchronize()
+    for l, X, W, s, h, Y in outs:
+        rows = _sampled_rows(l.T, 16, l.seed) if T > 1000 else np.arange(T)
+        ref = oracle.spmm(X.numpy()[rows], W.numpy(), l.N, l.M, scale=s.numpy())
+        assert np.array_equal(Y.cpu().numpy()[rows].view(np.uint32), ref.view(np.uint32)), l.name
+
+
+# --------------------------------------------------------------------------- edge cases and errors
+
+
+def test_t_zero_is_noop():
+    h = nm.nm_compress(_weights("int8", 64, 64, 1).cuda(), 2, 4)
+    X = torch.empty((0, 64), dtype=torch.int8, device="cuda")
+    Y = nm.nm_spmm(h, X)
+    assert Y.shape == (0, 64)
+
+
+def test_spmm_rejects_unaligned_and_unsupported():
+    h = nm.nm_compress(_weights("int8", 64, 64, 1).cuda(), 2, 4)
+    buf = torch.zeros(64 * 64 + 16, dtype=torch.int8, device="cuda")
+    Y = torch.empty((64, 64), dtype=torch.int32, device="cuda")
+    L = nm.lib()
+    assert L.nm_spmm(h.raw, buf.data_ptr() + 1, 64, Y.data_ptr(), None, None) == nm.NM_ERR_INVALID
+    assert L.nm_spmm(h.raw, buf.data_ptr(), -1, Y.data_ptr(), None, None) == nm.NM_ERR_INVALID
+    h8 = nm.nm_compress(_weights("int8", 16, 8, 1).cuda(), 2, 4)  # k = 8 bytes per row: not TMA-able
+    assert L.nm_spmm(h8.raw, buf.data_ptr(), 4, Y.data_ptr(), None, None) == nm.NM_ERR_UNSUPPORTED
+    assert "multiple of 16" in nm.nm_last_error()
+
+
+def test_output_canaries_untouched():
+    """Ragged tiles must not write past Y (guard elements after the output)."""
+    W = _weights("int8", 200, 784, 3)
+    X = _acts("int8", 77, 784, 4)
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    buf = torch.full((77 * 200 + 4096,), -7, dtype=torch.int32, device="cuda")
+    Y = buf[: 77 * 200].view(77, 200)
+    nm.nm_spmm(h, X.cuda(), Y=Y)
+    assert (buf[77 * 200:] == -7).all()
+    assert np.array_equal(Y.cpu().numpy(), oracle.spmm(X.numpy(), W.numpy(), 2, 4))
