@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the N:M sparse GEMM path on B200.
+
+One step = the whole path over the ViT-B/16 INT8 linear-layer set at batch 64
+(T = 12608 tokens; QKV 768->2304, proj 768->768, FC1 768->3072, FC2 3072->768;
+N:M in {1:4, 2:4, 2:8, 4:8}; per-output-channel fp32 scale, fp32 Y):
+for each of the 16 (layer, N:M) problems, re-pack the layer's weight
+(nm_recompress: top-N select + packed operand image) and run nm_spmm.
+Inputs are seeded synthetic tensors with the workload's shapes and value
+distributions (structured_sparse_gemm_compress_b200.inputs); every step
+streams about 1.7 GB, far more than the 126 MB L2, so no repeat is L2-warm.
+
+Metric: dense-equivalent TOPS = sum(2*T*K*n_out) / time, whole job (all ranks).
+Multi-GPU: replicas only -- tokens are independent, each rank runs its own
+batch on its own GPU with no data-path collective (weak scaling); the barrier
+and the max-over-ranks timing use torch.distributed.
+
+`--impl reference` times the CPU oracle (the only reference implementation
+there is) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from structured_sparse_gemm_compress_b200 import inputs  # noqa: E402
+
+METRIC = "N:M SpMM effective TOPS (dense-equiv) on ViT-B layers; % of sparse-TC roofline"
+UNIT = "TOPS"
+WORKLOAD = "ViT-B/16 INT8 linear set, batch 64 (T=12608), N:M in {1:4,2:4,2:8,4:8}, per-channel fp32 scale"
+CPU_SAMPLE_ROWS = 1536      # about 10-30 s of oracle work on the host cores
+REF_SAMPLE_ROWS = 192       # per reference-arm step, so --steps 20 stays within a few minutes
+
+
+_ONLY: list[str] = []
+
+
+def layers():
+    """The 16 (layer, N:M) problems, or the subset named by --only (name/N:M)."""
+    ls = inputs.vit_b_int8()
+    if _ONLY:
+        ls = [l for l in ls if f"{l.name}/{l.nm}" in _ONLY]
+        if not ls:
+            raise SystemExit(f"--only matched no problem: {_ONLY}")
+    return ls
+
+
+def alg_bytes(l) -> int:
+    """Algorithmic bytes of one SpMM launch: X + packed W (kept values + log2(M)
+    bits of position each) + Y + scale."""
+    import math
+    kept = l.n_out * (l.K // l.M) * l.N
+    wbytes = kept + (kept * math.ceil(math.log2(l.M)) + 7) // 8 if l.N != l.M else l.n_out * l.K
+    ybytes = l.T * l.n_out * 4
+    return l.T * l.K + wbytes + ybytes + (4 * l.n_out if l.scaled else 0)
+
+
+def pack_bytes(l) -> int:
+    """Algorithmic bytes of one re-pack: read W, write canonical values + positions."""
+    kept = l.n_out * (l.K // l.M) * l.N
+    return l.n_out * l.K + kept + (kept + 1) // 2
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        busy = [s for s in sm if s > 0.5 * max(mx or [1])] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- multi-rank plumbing
+
+
+def rank_env() -> tuple[int, int, int]:
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 without it)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time: replicas finish together only when the slowest does."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(ops_per_rank_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes its own batch (weak scaling)."""
+    return ops_per_rank_step * steps * world / (ms * 1e-3) / 1e12
+
+
+# --------------------------------------------------------------------------- reference arm (CPU oracle)
+
+
+def cpu_oracle_run(ls, rows: int):
+    """Oracle over a sample: the first `rows` tokens of every problem (compress,
+    decompress, triple-loop GEMM).  Returns (seconds, dense-equivalent ops)."""
+    import oracle
+
+    data = []
+    for l in ls:
+        W = l.weight().numpy()
+        X = l.activation(T=rows).numpy()
+        s = l.scale().numpy()
+        data.append((l, W, X, s))
+    t0 = time.perf_counter()
+    ops = 0
+    for l, W, X, s in data:
+        oracle.spmm(X, W, l.N, l.M, scale=s)
+        ops += 2 * rows * l.K * l.n_out
+    return time.perf_counter() - t0, ops
+
+
+def run_reference(args, rank: int) -> None:
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    ls = layers()
+    for _ in range(args.warmup):
+        cpu_oracle_run(ls, 16)
+    secs, ops = 0.0, 0
+    rows = args.cpu_rows or REF_SAMPLE_ROWS
+    for _ in range(args.steps):
+        s, o = cpu_oracle_run(ls, rows)
+        secs += s
+        ops += o
+    value = ops / secs / 1e12
+    sample = (f"first {rows} of 12608 tokens of each of the 16 (layer, N:M) problems per step "
+              f"(compress + decompress + triple-loop GEMM), {args.steps} steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+        "data": "synthetic", "config": {"workload": WORKLOAD + " (CPU oracle on a token sample)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="nm", choices=["nm", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", action="append", default=[],
+                    help="restrict to problems like vitb.fc1/2:4 (profiling a single kernel shape)")
+    args = ap.parse_args()
+    _ONLY.extend(args.only)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local_rank = rank_env()
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import structured_sparse_gemm_compress_b200 as nm
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    ls = layers()
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+
+    # Host-side inputs (pinned) and device buffers.  Weights and activations are
+    # shared by the four N:M variants of a layer; each problem has its own Y.
+    host = {}
+    for l in ls:
+        if l.name not in host:
+            host[l.name] = {"W": l.weight().pin_memory(), "X": l.activation().pin_memory(),
+                            "s": l.scale().pin_memory()}
+    devb = {n: {k: v.to(dev, non_blocking=True) for k, v in d.items()} for n, d in host.items()}
+    handles, Ys = [], []
+    for l in ls:
+        handles.append(nm.nm_compress(devb[l.name]["W"], l.N, l.M))
+        Ys.append(torch.empty((l.T, l.n_out), dtype=torch.float32, device=dev))
+    torch.cuda.synchronize()
+
+    def step(events=None):
+        for i, l in enumerate(ls):
+            d = devb[l.name]
+            if events is not None:
+                events[i][0].record(stream)
+            nm.nm_recompress(handles[i], d["W"], stream=stream)
+            if events is not None:
+                events[i][1].record(stream)
+            nm.nm_spmm(handles[i], d["X"], Y=Ys[i], scale=d["s"], stream=stream)
+            if events is not None:
+                events[i][2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for h in handles:
+        if nm.nm_device_status(h) != nm.NM_OK:
+            raise RuntimeError(nm.nm_last_error())
+
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in ls] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for k in range(args.steps):
+            step(ev[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = max_over_ranks(start.elapsed_time(stop), dist, dev)
+    for h in handles:
+        if nm.nm_device_status(h) != nm.NM_OK:
+            raise RuntimeError(nm.nm_last_error())
+
+    ops_step = sum(l.dense_ops() for l in ls)
+    value = whole_job_tops(ops_step, args.steps, world, ms)
+
+    # Roofline of the dominant kernel (the SpMM), from the per-launch events.
+    spmm_ms = [ev[k][i][1].elapsed_time(ev[k][i][2]) for k in range(args.steps) for i in range(len(ls))]
+    pack_ms = [ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps) for i in range(len(ls))]
+    spmm_bytes = sum(alg_bytes(l) for l in ls) * args.steps
+    pk = peaks()
+    achieved = spmm_bytes / (sum(spmm_ms) * 1e-3) / 1e9
+    per_layer = {}
+    for i, l in enumerate(ls):
+        t = statistics.median(ev[k][i][1].elapsed_time(ev[k][i][2]) for k in range(args.steps))
+        per_layer[f"{l.name}/{l.nm}"] = {"us": round(t * 1e3, 2), "dense_eq_tops": round(l.dense_ops() / t / 1e9, 1),
+                                        "gbs": round(alg_bytes(l) / t / 1e6, 1)}
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "spmm_vitb_int8_traffic.json")
+    if os.path.exists(tfile):
+        tj = json.load(open(tfile))
+        if tj.get("kernel_source_sha") == _kernel_sha():
+            traffic = tj.get("bytes_per_launch")
+
+    # cuBLAS dense INT8 GEMM of the same shapes (context: torch._int_mm -> int32).
+    cublas = {}
+    if rank == 0:
+        for name in sorted({x.name for x in ls}):
+            l = next(x for x in ls if x.name == name)
+            Xd, Wd = devb[name]["X"], devb[name]["W"]
+            Wt = Wd.t()
+            for _ in range(3):
+                torch._int_mm(Xd, Wt)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(10):
+                torch._int_mm(Xd, Wt)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / 10
+            cublas[name] = {"us": round(t * 1e3, 2), "dense_tops": round(l.dense_ops() / t / 1e9, 1)}
+
+    # End to end through the public API with host buffers: every step copies its
+    # inputs (weights, activations, scales) from pinned host memory and reads
+    # every output back.
+    e2e = None
+    if not args.no_e2e:
+        yh = [torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True) for Y in Ys]
+        h2d = sum(t.numel() * t.element_size() for d in host.values() for t in d.values())
+        d2h = sum(y.numel() * y.element_size() for y in yh)
+        e_steps = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            for n, d in host.items():
+                for key, t in d.items():
+                    devb[n][key].copy_(t, non_blocking=True)
+            step()
+            for y, Y in zip(yh, Ys):
+                y.copy_(Y, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(a.elapsed_time(b), dist, dev)
+        e2e = {"value": whole_job_tops(ops_step, e_steps, world, ems), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        oracle.build()
+        rows = args.cpu_rows or CPU_SAMPLE_ROWS
+        secs, ops = cpu_oracle_run(ls, rows)
+        cpu = {"value": ops / secs / 1e12, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+               "sample": f"first {rows} of 12608 tokens of each of the 16 (layer, N:M) problems "
+                         f"(compress + decompress + triple-loop GEMM), {secs:.1f} s"}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    launches = 2 * len(ls) * args.steps  # one pack + one SpMM kernel per problem per step
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": WORKLOAD if not _ONLY else f"{WORKLOAD}; only {','.join(_ONLY)}",
+                   "global_batch_tokens": 12608 * world, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: each step streams ~1.7 GB",
+                   "step": "per (layer, N:M): nm_recompress + nm_spmm"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "kernel": "spmm_kernel (all 16 launches of a step)", "peak_source": pk["source"]},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "spmm_only_tops": ops_step * args.steps / (sum(spmm_ms) * 1e-3) / 1e12,
+        "pack_us_per_step": 1e3 * sum(pack_ms) / args.steps,
+        "per_layer": per_layer,
+        "cublas_int8_dense": cublas,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _kernel_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("nm_spmm.cu", "nm_device.cuh"):
+        h.update(open(os.path.join(ROOT, "structured_sparse_gemm_compress_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    main()

@@ -83,6 +83,20 @@ def test_compress_format_and_image_bit_exact(dtype, N, M, n_out, K):
     assert np.array_equal(_np(Wm, dtype), ref_Wm)
 
 
+@pytest.mark.parametrize("N,M", [(2, 4), (4, 8)])
+def test_recompress_updates_in_place(N, M):
+    W1 = _weights("int8", 200, 512, seed=61)
+    W2 = _weights("int8", 200, 512, seed=62)
+    X = _acts("int8", 90, 512, seed=63)
+    h = nm.nm_compress(W1.cuda(), N, M)
+    nm.nm_recompress(h, W2.cuda())
+    values, idx = nm.nm_export(h)
+    ref_v, ref_i = oracle.compress(W2.numpy(), N, M)
+    assert np.array_equal(values.numpy(), ref_v) and np.array_equal(idx.numpy(), ref_i)
+    Y = nm.nm_spmm(h, X.cuda())
+    assert np.array_equal(Y.cpu().numpy(), oracle.spmm(X.numpy(), W2.numpy(), N, M))
+
+
 def test_hand_examples_on_gpu():
     g = json.load(open(GOLDEN))
     W = torch.zeros((4, 16), dtype=torch.int8)
