@@ -73,6 +73,34 @@ nm_status nm_compress(const void* W_dev, int64_t n_out, int64_t k, nm_dtype dt, 
                       void* stream, nm_handle** out);
 
 /*
+ * nm_spmm_noalloc -- the same product as nm_spmm for callers that cannot
+ * allocate device memory.  (The paper has no counterpart: this is a
+ * deployment variant.)  Such callers include serving engines that hand
+ * nearly all of HBM to their own pool up front, so a library cudaMalloc would
+ * fail, and latency-critical code that must not call cudaMalloc/cudaFree,
+ * which can synchronise the device and take a process-wide lock.
+ *
+ * Arguments, layouts, rounding and results are those of nm_spmm.  The
+ * difference is where the split-K scratch (partial tiles and per-tile arrival
+ * counters) lives: in one fixed array inside the library, 4 MiB of partials
+ * plus 1024 counters.  Every GPU that loads the library holds that array until
+ * the process exits.  This call never calls cudaMalloc, cudaFree or any
+ * allocating routine.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (set-up, once per device, with that device
+ *     current); make that first call before any stream capture.
+ *   - A shape whose split-K plan needs more than the array holds is rejected
+ *     with NM_ERR_UNSUPPORTED and a message naming the sizes; nm_spmm handles
+ *     it instead.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call clears the counters it uses (an asynchronous memset on `stream`).
+ *     Calls whose kernels overlap on the GPU (different streams, or different
+ *     host threads) race on the array: order them.
+ */
+nm_status nm_spmm_noalloc(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
+                          const float* scale_dev, void* stream);
+
+/*
  * nm_recompress -- prune and pack a new weight of the handle's shape, dtype and
  * N:M into the handle's existing device buffers (a weight update; same rule
  * and layouts as nm_compress).  Allocates nothing; stream-ordered, so an

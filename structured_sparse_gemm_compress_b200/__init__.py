@@ -24,7 +24,7 @@ _TORCH_DT = {torch.int8: NM_INT8, torch.float16: NM_FP16, torch.bfloat16: NM_BF1
 _ELEM = {NM_INT8: torch.int8, NM_FP16: torch.float16, NM_BF16: torch.bfloat16}
 
 # Every symbol include/nmspmm.h declares.
-EXPORTS = ("nm_compress", "nm_recompress", "nm_spmm", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
+EXPORTS = ("nm_compress", "nm_recompress", "nm_spmm", "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
            "nm_device_status", "nm_destroy", "nm_last_error", "nm_version", "nm_test_spmm_skip_stage")
 
 
@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
         L.nm_compress.argtypes = [vp, i64, i64, i32, i32, i32, vp, ctypes.POINTER(vp)]
         L.nm_recompress.argtypes = [vp, vp, vp]
         L.nm_spmm.argtypes = [vp, vp, i64, vp, vp, vp]
+        L.nm_spmm_noalloc.argtypes = [vp, vp, i64, vp, vp, vp]
         L.nm_test_spmm_skip_stage.argtypes = [vp, vp, i64, vp, vp, vp, i32, i64]
         L.nm_decompress.argtypes = [vp, vp, vp]
         L.nm_export.argtypes = [vp, vp, vp]
@@ -60,7 +61,7 @@ def lib() -> ctypes.CDLL:
         L.nm_destroy.restype = None
         L.nm_last_error.restype = ctypes.c_char_p
         L.nm_version.restype = ctypes.c_char_p
-        for name in ("nm_compress", "nm_recompress", "nm_spmm", "nm_test_spmm_skip_stage", "nm_decompress", "nm_export",
+        for name in ("nm_compress", "nm_recompress", "nm_spmm", "nm_spmm_noalloc", "nm_test_spmm_skip_stage", "nm_decompress", "nm_export",
                      "nm_export_sizes", "nm_query", "nm_device_status"):
             getattr(L, name).restype = i32
         _lib = L
@@ -154,6 +155,14 @@ def nm_spmm(h: NMHandle, X: torch.Tensor, Y: torch.Tensor | None = None, scale: 
     if scale is not None and (scale.dtype != torch.float32 or scale.numel() != h.n_out or not scale.is_cuda):
         raise ValueError("scale must be a CUDA float32 tensor of n_out elements")
     _check(lib().nm_spmm(h.raw, _ptr(X), T, _ptr(Y), _ptr(scale), _stream(stream)))
+    return Y
+
+
+def nm_spmm_noalloc(h: NMHandle, X: torch.Tensor, Y: torch.Tensor, scale: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """nm_spmm for callers that cannot allocate: split-K scratch lives in a fixed
+    array inside the library (limits and ordering rules in include/nmspmm.h)."""
+    _check(lib().nm_spmm_noalloc(h.raw, _ptr(X), X.shape[0], _ptr(Y), _ptr(scale), _stream(stream)))
     return Y
 
 

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 
@@ -216,6 +217,35 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   return NM_OK;
 }
 
+// ---- scratch of the allocation-free entry point (nm_spmm_noalloc)
+//
+// A fixed, file-scope device array instead of cudaMalloc: 4 MiB of split-K
+// partial tiles followed by 1024 per-tile arrival counters.  Every GPU that
+// loads this library holds it until the process exits.  Host code may not use
+// the array's name as an address (on the host it is only a stand-in), so the
+// first call on each device looks its device address up with
+// cudaGetSymbolAddress while that device is current, and passes that address
+// to the kernel.
+constexpr size_t kNoAllocPartialBytes = size_t(4) << 20;
+constexpr int kNoAllocCounters = 1024;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocPartialBytes + kNoAllocCounters * sizeof(int)];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+nm_status noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= 64) return fail(NM_ERR_UNSUPPORTED, "device index %d above 63", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "look up the device address of the static split-K scratch");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return NM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -357,6 +387,65 @@ nm_status nm_device_status(const nm_handle* h) {
   static const char* where[] = {"", "producer waiting for a free stage", "MMA waiting for a free accumulator",
                                 "MMA waiting for operands", "epilogue waiting for an accumulator"};
   return fail(NM_ERR_TIMEOUT, "a kernel gave up a bounded wait (%s)", (word >= 1 && word <= 4) ? where[word] : "?");
+}
+
+nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y, const float* scale,
+                          void* stream) {
+  g_err.clear();
+  nm_status st = check_handle(hc);
+  if (st != NM_OK) return st;
+  nm_handle* h = const_cast<nm_handle*>(hc);  // only the tensor-map cache (host memory) changes
+  void* scratch = nullptr;
+  st = noalloc_scratch(h->device, &scratch);  // first call on this device: address lookup
+  if (st != NM_OK) return st;
+  if (T < 0) return fail(NM_ERR_INVALID, "T must be >= 0 (got %lld)", (long long)T);
+  if (T == 0) return NM_OK;
+  if (!X || !Y) return fail(NM_ERR_INVALID, "null X or Y");
+  if (T > INT32_MAX) return fail(NM_ERR_UNSUPPORTED, "T above 2^31-1");
+  const int es = nm::elem_bytes(h->dt);
+  if (!aligned(X, 16) || !aligned(Y, 16)) return fail(NM_ERR_INVALID, "X and Y must be 16-byte aligned");
+  if ((h->k * es) % 16 != 0)
+    return fail(NM_ERR_UNSUPPORTED, "k * sizeof(dtype) must be a multiple of 16 bytes (k=%lld)", (long long)h->k);
+  if (scale && !aligned(scale, 4)) return fail(NM_ERR_INVALID, "scale must be 4-byte aligned");
+  const size_t ybytes = (size_t)T * h->n_out * ((h->dt == nm::DT_I8) ? 4 : 2);
+  const size_t xbytes = (size_t)T * h->k * es;
+  const uintptr_t xs = (uintptr_t)X, ys = (uintptr_t)Y;
+  if (xs < ys + ybytes && ys < xs + xbytes) return fail(NM_ERR_INVALID, "Y overlaps X");
+
+  const nm::Plan p = make_plan(h, T, num_sms(h->device));
+  st = make_x_map(h, X, T, p.bn);
+  if (st != NM_OK) return st;
+  nm::SpmmArgs a{};
+  a.bpack = h->d_bpack;
+  a.Y = Y;
+  a.scale = scale;
+  a.err = h->d_err;
+  a.T = (int)T;
+  a.n_out = (int)h->n_out;
+  a.n_kb = h->n_kb;
+  a.n_ct = h->n_ct;
+  a.n_tt = p.n_tt;
+  a.splits = p.splits;
+  a.kb_per_split = p.kb_per_split;
+  a.units = p.units;
+  a.timeout_ns = 1000000000ull;
+  a.inject_skip = -1;
+  if (p.splits > 1) {
+    const int tiles = h->n_ct * p.n_tt;
+    const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
+    if (need > kNoAllocPartialBytes || tiles > kNoAllocCounters)
+      return fail(NM_ERR_UNSUPPORTED,
+                  "this shape needs %zu bytes of split-K scratch for %d tiles; the allocation-free entry point "
+                  "holds at most %zu bytes and %d tiles (use nm_spmm)",
+                  need, tiles, kNoAllocPartialBytes, kNoAllocCounters);
+    a.ws = scratch;
+    a.cnt = reinterpret_cast<int*>(static_cast<unsigned char*>(scratch) + kNoAllocPartialBytes);
+    // The array keeps the previous call's contents: the counters must start at zero.
+    cudaError_t e = cudaMemsetAsync(a.cnt, 0, (size_t)tiles * sizeof(int), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "clear the split-K counters");
+  }
+  cudaError_t e = nm::launch_spmm(h, &h->tm, p, a, (cudaStream_t)stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch SpMM kernel");
 }
 
 void nm_destroy(nm_handle* h) {
