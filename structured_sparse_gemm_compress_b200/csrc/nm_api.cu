@@ -15,7 +15,7 @@
 #include <new>
 #include <string>
 
-#include "../../include/nmspmm.h"
+#include "nmspmm.h"
 #include "nm_device.cuh"
 #include "nm_internal.h"
 
@@ -102,6 +102,69 @@ nm_status make_x_map(nm_handle* h, const void* X, int64_t T, int bn) {
   return NM_OK;
 }
 
+// The packed operand image as a 2-D tensor of 128-byte rows, so one tensor
+// copy with a box of (chunk bytes / 128) rows brings one chunk (values and
+// positions together) into shared memory.
+nm_status make_w_map(nm_handle* h) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t rows = (cuuint64_t)(h->bpack_bytes / 128);
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, (cuuint32_t)(h->chunk / 128)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&h->tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, h->d_bpack, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for the packed image", (int)r);
+  h->has_tmw = 1;
+  return NM_OK;
+}
+
+// Output Y [T][n_out] as a 2-D tensor for the epilogue's TMA stores: box =
+// 32 channels x ch tokens, no swizzle; stores outside the tensor are clipped.
+// Returns false (direct stores instead) when the row pitch is not a multiple of
+// 16 bytes, which TMA requires.
+bool make_y_map(nm_handle* h, void* Y, int64_t T, int out_es, int out_ty, int ch, nm_status* st) {
+  *st = NM_OK;
+  if ((h->n_out * out_es) % 16 != 0) return false;
+  const int key = out_ty * 1024 + ch;
+  if (h->tmy_y == Y && h->tmy_T == T && h->tmy_out == key) return true;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    *st = fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)h->n_out, (cuuint64_t)T};
+  cuuint64_t strides[1] = {(cuuint64_t)(h->n_out * out_es)};
+  cuuint32_t box[2] = {32, (cuuint32_t)ch};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&h->tmy, (CUtensorMapDataType)out_ty, 2, Y, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    h->tmy_y = nullptr;
+    *st = fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for the output", (int)r);
+    return false;
+  }
+  h->tmy_y = Y;
+  h->tmy_T = T;
+  h->tmy_out = key;
+  return true;
+}
+
+// Output element type and size of a launch: int32 / fp32 for INT8 (without /
+// with scale), else the input's 16-bit type.
+void out_type(const nm_handle* h, bool scaled, int* es, int* ty) {
+  if (h->dt == nm::DT_I8) {
+    *es = 4;
+    *ty = scaled ? (int)CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : (int)CU_TENSOR_MAP_DATA_TYPE_INT32;
+  } else {
+    *es = 2;
+    *ty = h->dt == nm::DT_F16 ? (int)CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : (int)CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  }
+}
+
 // Adaptive parallelism: pick the token tile and split-K factor for this shape.
 // Token tile: minimise (waves of persistent CTAs) x (per-tile cost ~ bn + 32).
 // Split-K: only when even the smallest tile leaves most SMs idle; partials are
@@ -111,6 +174,24 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms) {
   nm::Plan p;
   const int forced_bn = env_int("NMSPMM_FORCE_BN", 0);
   const int forced_split = env_int("NMSPMM_FORCE_SPLITK", 0);
+  const int forced_xs = env_int("NMSPMM_FORCE_XS", -1);  // -1 auto, 0 off, 1 on when eligible
+  const int forced_grid = env_int("NMSPMM_FORCE_GRID", 0);  // cap on persistent CTAs (tests, sweeps)
+  if (forced_grid > 0) sms = std::min(sms, forced_grid);
+  // X-stationary mode: INT8 with at most kXsMaxKb k-blocks, several channel tiles
+  // sharing each X tile, and enough 128-token tiles to fill the SMs without split-K.
+  const int64_t tt128 = (T + 127) / 128;
+  const bool xs_ok = h->dt == nm::DT_I8 && h->n_kb <= nm::kXsMaxKb && (forced_bn == 0 || forced_bn == 128) &&
+                     forced_split <= 1 && h->n_ct >= 2;
+  if (xs_ok && (forced_xs == 1 || (forced_xs == -1 && tt128 * h->n_ct >= 2 * sms))) {
+    p.bn = 128;
+    p.xkb = h->n_kb;
+    p.n_tt = (int)tt128;
+    p.splits = 1;
+    p.kb_per_split = h->n_kb;
+    p.units = (int)(tt128 * h->n_ct);
+    p.grid = std::min(p.units, sms);
+    return p;
+  }
   const int bns[3] = {128, 64, 32};
   double best = 1e300;
   for (int bn : bns) {
@@ -187,6 +268,11 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   a.units = p.units;
   a.timeout_ns = timeout_ns;
   a.inject_skip = inject_skip;
+  a.w_tma = (h->has_tmw && env_int("NMSPMM_W_BULK", 0) == 0) ? 1 : 0;
+#ifdef NM_TRACE
+  // timeline builds only: device buffer of grid * kTraceStride int64 given as an integer address
+  if (const char* tp = getenv("NMSPMM_TRACE_PTR")) a.trace = reinterpret_cast<long long*>(strtoull(tp, nullptr, 0));
+#endif
   if (p.splits > 1) {
     const int tiles = h->n_ct * p.n_tt;
     const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
@@ -212,7 +298,11 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
     a.ws = h->d_ws;
     a.cnt = h->d_cnt;
   }
-  cudaError_t e = nm::launch_spmm(h, &h->tm, p, a, (cudaStream_t)stream);
+  int oes, oty;
+  out_type(h, scale != nullptr, &oes, &oty);
+  a.tma_store = make_y_map(h, Y, T, oes, oty, std::min(32, p.bn / 2), &st) ? 1 : 0;
+  if (st != NM_OK) return st;
+  cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "launch SpMM kernel");
   return NM_OK;
 }
@@ -299,6 +389,8 @@ nm_status nm_compress(const void* W_dev, int64_t n_out, int64_t k, nm_dtype dt, 
     st = cuda_fail(e, "clear error word");
   else if ((e = nm::launch_compress(h, W_dev, (cudaStream_t)stream)) != cudaSuccess)
     st = cuda_fail(e, "launch compress kernel");
+  else
+    st = make_w_map(h);
   if (st != NM_OK) {
     const std::string msg = g_err;
     nm_destroy(h);
@@ -430,6 +522,7 @@ nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y
   a.units = p.units;
   a.timeout_ns = 1000000000ull;
   a.inject_skip = -1;
+  a.w_tma = h->has_tmw;
   if (p.splits > 1) {
     const int tiles = h->n_ct * p.n_tt;
     const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
@@ -444,7 +537,11 @@ nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y
     cudaError_t e = cudaMemsetAsync(a.cnt, 0, (size_t)tiles * sizeof(int), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "clear the split-K counters");
   }
-  cudaError_t e = nm::launch_spmm(h, &h->tm, p, a, (cudaStream_t)stream);
+  int oes, oty;
+  out_type(h, scale != nullptr, &oes, &oty);
+  a.tma_store = make_y_map(h, Y, T, oes, oty, std::min(32, p.bn / 2), &st) ? 1 : 0;
+  if (st != NM_OK) return st;
+  cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch SpMM kernel");
 }
 

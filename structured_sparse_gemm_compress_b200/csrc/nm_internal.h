@@ -36,6 +36,14 @@ struct nm_handle {
   int64_t tm_T = -1;
   int tm_bn = 0;
   alignas(64) CUtensorMap tm;
+  // the packed image as a 2-D tensor of 128-byte rows (one box = one chunk)
+  int has_tmw = 0;
+  alignas(64) CUtensorMap tmw;
+  // cached tensor map of the last output seen
+  const void* tmy_y = nullptr;
+  int64_t tmy_T = -1;
+  int tmy_out = -1;
+  alignas(64) CUtensorMap tmy;
 };
 
 namespace nm {
@@ -48,7 +56,11 @@ struct Plan {
   int n_tt = 1;       // token tiles
   int units = 1;      // (tile, split) work units
   int grid = 1;       // persistent CTAs
+  int xkb = 0;        // > 0: X-stationary mode holding this many k-blocks of X resident
 };
+
+// Largest number of INT8 k-blocks (256 dense k each) the X-stationary mode keeps resident.
+constexpr int kXsMaxKb = 3;
 
 struct SpmmArgs {
   const uint8_t* bpack;
@@ -59,13 +71,21 @@ struct SpmmArgs {
   int* err;
   int T, n_out, n_kb, n_ct, n_tt, splits, kb_per_split, units;
   unsigned long long timeout_ns;
+  int tma_store;      // 1: epilogue writes Y with TMA tensor stores (tmY valid)
+  int w_tma;          // 1: packed chunks arrive by 2-D tensor copy (tmW valid), else one bulk copy
   int inject_skip;    // test hook: producer omits the stage with this index (-1: never)
+  long long* trace;   // timeline buffer, only written by builds compiled with NM_TRACE
 };
+
+// Timeline trace layout (builds with NM_TRACE): per CTA kTraceStride int64
+// slots: [kind][index], kinds below, kTraceMax indices each.
+constexpr int kTraceMax = 64;
+enum : int { TR_P_ISSUE = 0, TR_M_FULL, TR_M_DONE, TR_M_ACCE, TR_E_START, TR_E_END, TR_KINDS };
+constexpr int kTraceStride = TR_KINDS * kTraceMax;
 
 cudaError_t launch_compress(const nm_handle* h, const void* W, cudaStream_t s);
 cudaError_t launch_decompress(const nm_handle* h, void* Wout, cudaStream_t s);
-cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a,
-                        cudaStream_t s);
-size_t spmm_smem_bytes(int dt, int img, int bn);
+cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const CUtensorMap* tmY, const Plan& p,
+                        const SpmmArgs& a, cudaStream_t s);
 
 }  // namespace nm

@@ -50,70 +50,145 @@ __device__ __forceinline__ void unpack16(uint4 q, T* v) {
   }
 }
 
-// Kept-position mask of one group of M: N rounds of "largest magnitude not yet
-// taken, first position on ties".
-template <int DT>
-__device__ __forceinline__ uint32_t select_group(const uint32_t* a, int N, int M) {
+// Kept-position mask of one group of M (compile-time N, M, fully unrolled):
+// N rounds of "largest magnitude not yet taken, first position on ties".
+template <int DT, int N, int M>
+__device__ __forceinline__ uint32_t select_group(const typename Elem<DT>::T* v) {
   uint32_t keep = 0;
+#pragma unroll
   for (int j = 0; j < N; ++j) {
-    int best = -1;
+    int best = 0;
     uint32_t bv = 0;
+    bool found = false;
+#pragma unroll
     for (int p = 0; p < M; ++p) {
-      if ((keep >> p) & 1u) continue;
-      if (best < 0 || a[p] > bv) {
-        best = p;
-        bv = a[p];
-      }
+      const uint32_t a = Elem<DT>::mag(v[p]);
+      const bool avail = ((keep >> p) & 1u) == 0u;
+      const bool better = avail && (!found || a > bv);
+      best = better ? p : best;
+      bv = better ? a : bv;
+      found = found || avail;
     }
     keep |= 1u << best;
   }
   return keep;
 }
 
-template <int DT>
+// v[p] for a runtime p in [0, M), without indexing a register array dynamically.
+template <int M, typename T>
+__device__ __forceinline__ T pick(const T* v, int p) {
+  T out = v[0];
+#pragma unroll
+  for (int q = 1; q < M; ++q) out = (p == q) ? v[q] : out;
+  return out;
+}
+
+// Store `bytes` (4, 8, 16 or 32) bytes held in w[] at dst: one vector store
+// when dst is aligned to it, else byte stores.
+__device__ __forceinline__ void store_bytes(uint8_t* dst, const uint32_t* w, int bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(dst);
+  if (bytes == 32 && (a & 15u) == 0) {
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  } else if (bytes == 16 && (a & 15u) == 0) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if (bytes == 8 && (a & 7u) == 0) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+  } else if (bytes == 4 && (a & 3u) == 0) {
+    *reinterpret_cast<uint32_t*>(dst) = w[0];
+  } else {
+    for (int b = 0; b < bytes; ++b) dst[b] = (uint8_t)(w[b >> 2] >> (8 * (b & 3)));
+  }
+}
+
+template <int DT, int N, int M>
 __global__ void __launch_bounds__(256) compress_kernel(const typename Elem<DT>::T* __restrict__ W, int64_t n_out,
-                                                       int64_t K, int N, int M, int img, int n_kb,
-                                                       typename Elem<DT>::T* __restrict__ values,
+                                                       int64_t K, int n_kb, typename Elem<DT>::T* __restrict__ values,
                                                        uint8_t* __restrict__ idx, int64_t idx_pitch,
                                                        uint8_t* __restrict__ bpack, int64_t total_units) {
   using T = typename Elem<DT>::T;
   constexpr int KB = kblock_elems(DT);
   constexpr int ES = elem_bytes(DT);
+  constexpr int IMG = (N == M || (N == 4 && M == 8)) ? IMG_DENSE : IMG_SP24;
+  constexpr int G = 16 / M;            // groups of M in one 16-position unit
+  constexpr int CNT = 16 * N / M;      // kept values of a full unit
   const int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (unit >= total_units) return;
   const int64_t units_per_row = (int64_t)n_kb * (KB / 16);
   const int64_t r = unit / units_per_row;
   const int64_t k0 = (unit - r * units_per_row) * 16;
 
+  // ---- load 16 positions (zero beyond the row or beyond K)
   T raw[16];
-  uint32_t a[16];
-  const bool row_ok = r < n_out;
   const int64_t rem = K - k0;
-  const int valid = row_ok ? (int)(rem < 0 ? 0 : (rem > 16 ? 16 : rem)) : 0;
+  const int valid = r < n_out ? (int)(rem < 0 ? 0 : (rem > 16 ? 16 : rem)) : 0;
+  const T* src = W + r * K + k0;
+  if (valid == 16 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    raw[c] = (c < valid) ? W[r * K + k0 + c] : (T)0;
-    a[c] = Elem<DT>::mag(raw[c]);
+    for (int h = 0; h < ES; ++h) unpack16<T>(__ldg(reinterpret_cast<const uint4*>(src) + h), raw + h * (16 / ES));
+  } else {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) raw[c] = (c < valid) ? src[c] : (T)0;
   }
-  uint32_t keep = 0;
-  for (int g = 0; g < valid / M; ++g) keep |= select_group<DT>(a + g * M, N, M) << (g * M);
 
-  // ---- canonical format
+  uint32_t keep = 0;
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+    if (g * M < valid) keep |= select_group<DT, N, M>(raw + g * M) << (g * M);
+
+  // ---- canonical format: kept values in ascending position + 4-bit positions
   if (valid > 0) {
     const int64_t kept_per_row = (K / M) * N;
     const int64_t e0 = (k0 / M) * N;
-    T* vdst = values + r * kept_per_row + e0;
-    uint64_t nib = 0;
-    int cnt = 0;
-    for (int c = 0; c < valid; ++c) {
-      if ((keep >> c) & 1u) {
-        vdst[cnt] = raw[c];
-        nib |= (uint64_t)(c % M) << (4 * cnt);
-        ++cnt;
+    T vals[CNT];
+    uint32_t nib[CNT / 8 > 0 ? CNT / 8 : 1] = {};
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      uint32_t m = (keep >> (g * M)) & ((1u << M) - 1u);
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const int p = __ffs(m) - 1;  // j-th kept position of the group (ascending)
+        m &= m - 1u;
+        const int e = g * N + j;
+        vals[e] = pick<M>(raw + g * M, p < 0 ? 0 : p);
+        nib[e / 8] |= (uint32_t)(p & 0xF) << (4 * (e % 8));
       }
     }
+    uint8_t* vdst = reinterpret_cast<uint8_t*>(values + r * kept_per_row + e0);
     uint8_t* idst = idx + r * idx_pitch + e0 / 2;
-    for (int b = 0; b < (cnt + 1) / 2; ++b) idst[b] = (uint8_t)(nib >> (8 * b));
+    if (valid == 16) {
+      uint32_t vw[CNT * ES / 4 > 0 ? CNT * ES / 4 : 1];
+      if constexpr (CNT * ES >= 4) {
+#pragma unroll
+        for (int i = 0; i < CNT * ES / 4; ++i) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int b = 0; b < 4 / ES; ++b) {
+            const int e = i * (4 / ES) + b;
+            w |= (ES == 1 ? (uint32_t)(uint8_t)vals[e] : (uint32_t)(uint16_t)vals[e]) << (8 * ES * b);
+          }
+          vw[i] = w;
+        }
+        store_bytes(vdst, vw, CNT * ES);
+      }
+      if constexpr (CNT / 2 >= 4) {
+        store_bytes(idst, nib, CNT / 2);
+      } else {
+        for (int b = 0; b < CNT / 2; ++b) idst[b] = (uint8_t)(nib[0] >> (8 * b));
+      }
+    } else {  // ragged end of a row: only the groups that exist
+      const int cnt = (valid / M) * N;
+      T* vd = values + r * kept_per_row + e0;
+#pragma unroll
+      for (int e = 0; e < CNT; ++e)
+        if (e < cnt) vd[e] = vals[e];
+      for (int b = 0; b < (cnt + 1) / 2; ++b) {
+        const int e = 2 * b;
+        uint8_t byte = (uint8_t)((nib[e / 8] >> (4 * (e % 8))) & 0xF);
+        if (e + 1 < cnt) byte |= (uint8_t)(((nib[(e + 1) / 8] >> (4 * ((e + 1) % 8))) & 0xF) << 4);
+        idst[b] = byte;
+      }
+    }
   }
 
   // ---- packed operand image
@@ -121,41 +196,48 @@ __global__ void __launch_bounds__(256) compress_kernel(const typename Elem<DT>::
   const uint32_t rr = (uint32_t)(r % kRows);
   const int kb = (int)(k0 / KB);
   const uint32_t kk = (uint32_t)(k0 % KB);
-  uint8_t* chunk = bpack + ((size_t)ct * n_kb + kb) * (size_t)chunk_bytes(DT, img);
+  uint8_t* chunk = bpack + ((size_t)ct * n_kb + kb) * (size_t)chunk_bytes(DT, IMG);
 
-  if (img == IMG_SP24) {
+  if constexpr (IMG == IMG_SP24) {
     T comp[8];
     uint32_t meta = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 4; ++j) {  // groups of four: two slots each, positions ascending
       const uint32_t bits = (keep >> (4 * j)) & 0xFu;
+      const int n = __popc(bits);
+      const int lo = __ffs(bits) - 1;
+      const int hi = 31 - __clz(bits | 1u);
       int i0, i1;
       T v0, v1;
-      const int n = __popc(bits);
       if (n >= 2) {
-        i0 = __ffs(bits) - 1;
-        i1 = __ffs(bits & (bits - 1)) - 1;
-        v0 = raw[4 * j + i0];
-        v1 = raw[4 * j + i1];
+        i0 = lo; i1 = hi;
+        v0 = pick<4>(raw + 4 * j, lo);
+        v1 = pick<4>(raw + 4 * j, hi);
+      } else if (n == 1 && lo < 3) {
+        i0 = lo; i1 = 3;
+        v0 = pick<4>(raw + 4 * j, lo);
+        v1 = (T)0;
       } else if (n == 1) {
-        const int p = __ffs(bits) - 1;
-        if (p < 3) {
-          i0 = p; i1 = 3; v0 = raw[4 * j + p]; v1 = (T)0;
-        } else {
-          i0 = 0; i1 = 3; v0 = (T)0; v1 = raw[4 * j + 3];
-        }
+        i0 = 0; i1 = 3;
+        v0 = (T)0;
+        v1 = raw[4 * j + 3];
       } else {
-        i0 = 0; i1 = 1; v0 = (T)0; v1 = (T)0;
+        i0 = 0; i1 = 1;
+        v0 = (T)0;
+        v1 = (T)0;
       }
       comp[2 * j] = v0;
       comp[2 * j + 1] = v1;
       meta |= (uint32_t)(i0 | (i1 << 2)) << (4 * j);
     }
-    if (ES == 1) {
-      uint64_t packed = 0;
+    if constexpr (ES == 1) {
+      uint32_t w0 = 0, w1 = 0;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) packed |= (uint64_t)(uint8_t)comp[e] << (8 * e);
-      *reinterpret_cast<uint64_t*>(chunk + swz128(rr, kk / 2)) = packed;
+      for (int e = 0; e < 4; ++e) {
+        w0 |= (uint32_t)(uint8_t)comp[e] << (8 * e);
+        w1 |= (uint32_t)(uint8_t)comp[e + 4] << (8 * e);
+      }
+      *reinterpret_cast<uint2*>(chunk + swz128(rr, kk / 2)) = make_uint2(w0, w1);
     } else {
       *reinterpret_cast<uint4*>(chunk + swz128(rr, kk)) = pack16<T>(comp);
     }
@@ -231,29 +313,38 @@ __global__ void __launch_bounds__(256) decompress_kernel(const uint8_t* __restri
 
 }  // namespace
 
+template <int DT, int N, int M>
+static void launch_compress_t(const nm_handle* h, const void* W, int64_t total, cudaStream_t s) {
+  using T = typename Elem<DT>::T;
+  const int threads = 256;
+  const unsigned blocks = (unsigned)((total + threads - 1) / threads);
+  compress_kernel<DT, N, M><<<blocks, threads, 0, s>>>((const T*)W, h->n_out, h->k, h->n_kb, (T*)h->d_values,
+                                                       h->d_idx, h->idx_pitch, h->d_bpack, total);
+}
+
+template <int DT>
+static cudaError_t launch_compress_dt(const nm_handle* h, const void* W, int64_t total, cudaStream_t s) {
+  const int nm_code = h->N * 16 + h->M;
+  switch (nm_code) {
+    case 1 * 16 + 4: launch_compress_t<DT, 1, 4>(h, W, total, s); break;
+    case 2 * 16 + 4: launch_compress_t<DT, 2, 4>(h, W, total, s); break;
+    case 2 * 16 + 8: launch_compress_t<DT, 2, 8>(h, W, total, s); break;
+    case 4 * 16 + 8: launch_compress_t<DT, 4, 8>(h, W, total, s); break;
+    case 4 * 16 + 4: launch_compress_t<DT, 4, 4>(h, W, total, s); break;
+    case 8 * 16 + 8: launch_compress_t<DT, 8, 8>(h, W, total, s); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_compress(const nm_handle* h, const void* W, cudaStream_t s) {
   const int KB = kblock_elems(h->dt);
   const int64_t total = (int64_t)h->n_ct * kRows * ((int64_t)h->n_kb * (KB / 16));
-  const int threads = 256;
-  const unsigned blocks = (unsigned)((total + threads - 1) / threads);
   switch (h->dt) {
-    case DT_I8:
-      compress_kernel<DT_I8><<<blocks, threads, 0, s>>>(
-          (const int8_t*)W, h->n_out, h->k, h->N, h->M, h->img, h->n_kb, (int8_t*)h->d_values, h->d_idx,
-          h->idx_pitch, h->d_bpack, total);
-      break;
-    case DT_F16:
-      compress_kernel<DT_F16><<<blocks, threads, 0, s>>>(
-          (const uint16_t*)W, h->n_out, h->k, h->N, h->M, h->img, h->n_kb, (uint16_t*)h->d_values, h->d_idx,
-          h->idx_pitch, h->d_bpack, total);
-      break;
-    default:
-      compress_kernel<DT_BF16><<<blocks, threads, 0, s>>>(
-          (const uint16_t*)W, h->n_out, h->k, h->N, h->M, h->img, h->n_kb, (uint16_t*)h->d_values, h->d_idx,
-          h->idx_pitch, h->d_bpack, total);
-      break;
+    case DT_I8: return launch_compress_dt<DT_I8>(h, W, total, s);
+    case DT_F16: return launch_compress_dt<DT_F16>(h, W, total, s);
+    default: return launch_compress_dt<DT_BF16>(h, W, total, s);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_decompress(const nm_handle* h, void* Wout, cudaStream_t s) {

@@ -18,12 +18,16 @@
 // = token; the epilogue therefore stores 32 consecutive channels of one token
 // per warp instruction (128 B, coalesced) without a transpose.
 //
-// CTA = 6 warps, one persistent CTA per SM:
+// CTA = 10 warps, one persistent CTA per SM:
 //   warp 0      producer: one bulk copy of the packed weight chunk (values +
 //               positions) and two 2-D tensor copies of X per stage;
 //   warp 1      TMEM owner and MMA issuer (one thread): copies the positions
 //               into TMEM (tcgen05.cp) and issues tcgen05.mma(.sp);
-//   warps 2..5  epilogue: tcgen05.ld, optional per-channel scale, stores.
+//   warps 2..9  epilogue, two warps per TMEM lane quarter (one per half of the
+//               token columns): tcgen05.ld, optional per-channel scale, then
+//               either a staged tile in shared memory written by a TMA tensor
+//               store (3 instructions per element) or, when Y's row pitch is
+//               not a multiple of 16 bytes, direct coalesced stores.
 // Two TMEM accumulators let the epilogue of one tile overlap the mainloop of
 // the next.  Every wait is bounded; on a timeout the kernel records an error
 // word, drains its own copies and MMAs, frees TMEM and returns.
@@ -37,27 +41,52 @@ namespace nm {
 
 enum : int { OUT_I32 = 0, OUT_F32 = 1, OUT_F16 = 2, OUT_BF16 = 3 };
 
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemBudget = 227 * 1024 - 1024;  // dynamic shared memory after 1 KB alignment slack
 
-template <int DT, int IMG, int BN>
+constexpr int out_bytes(int out) { return (out == OUT_I32 || out == OUT_F32) ? 4 : 2; }
+
+// Kernel configuration.  XKB = 0: streaming mode, every stage carries a packed
+// weight chunk and the matching X boxes.  XKB > 0: X-stationary mode, the
+// whole X tile of a token tile (up to XKB k-blocks) stays resident in shared
+// memory while the CTA walks the channel tiles of its range; stages carry only
+// packed weight chunks, so X is read from L2 once per token tile instead of
+// once per 128-channel tile.
+template <int DT, int IMG, int BN, int OUT, int XKB>
 struct Cfg {
   static constexpr bool SP = IMG == IMG_SP24;
+  static constexpr bool XS = XKB > 0;
   static constexpr int KB = kblock_elems(DT);
   static constexpr int CHUNK = chunk_bytes(DT, IMG);
   static constexpr int B_BOX = BN * 128;            // one 128-byte-wide box of X rows
-  static constexpr int STAGE = CHUNK + 2 * B_BOX;   // multiple of 1024
-  static constexpr int STAGES = (kSmemBudget / STAGE) > 8 ? 8 : (kSmemBudget / STAGE);
+  static constexpr int B_KBLK = 2 * B_BOX;          // X bytes of one k-block
+  static constexpr int STAGE = XS ? CHUNK : CHUNK + B_KBLK;  // multiple of 1024
+  static constexpr int X_BYTES = XKB * B_KBLK;      // resident X region (X-stationary mode)
   static constexpr int MMAS = SP ? 4 : 8;           // MMAs per stage (each 32 B of A per row)
   static constexpr int E_COLS = SP ? (DT == DT_I8 ? 8 : 4) : 0;
   static constexpr int E_COL0 = 2 * BN;             // metadata slots after the two accumulators
   static constexpr int COLS_NEEDED = 2 * BN + 2 * E_COLS;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 : COLS_NEEDED <= 128 ? 128
                                    : COLS_NEEDED <= 256 ? 256 : 512;
-  static constexpr int SMEM = STAGES * STAGE + 1024;
-  static_assert(STAGE % 1024 == 0, "stage must keep 1024-byte alignment");
+  // epilogue: each warp owns BN/2 token columns of its lane quarter, in chunks of CH
+  static constexpr int HALF = BN / 2;
+  static constexpr int CH = HALF >= 32 ? 32 : HALF;
+  static constexpr int NCH = HALF / CH;
+  static constexpr int OES = out_bytes(OUT);
+  static constexpr int EPI_BUF = CH * 32 * OES;     // one staged [CH tokens][32 channels] tile
+  static constexpr int AVAIL = kSmemBudget - X_BYTES;
+  // two staging buffers per warp unless that would leave fewer stages than wanted
+  static constexpr int WANT = XS ? 4 : 3;
+  static constexpr int EPI_NB = (AVAIL - 2 * kEpiWarps * EPI_BUF) / STAGE >= WANT ? 2 : 1;
+  static constexpr int EPI_BYTES = EPI_NB * kEpiWarps * EPI_BUF;
+  static constexpr int STAGES_FIT = (AVAIL - EPI_BYTES) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int SMEM = STAGES * STAGE + X_BYTES + EPI_BYTES + 1024;
+  static_assert(STAGE % 1024 == 0 && B_KBLK % 1024 == 0, "stages keep 1024-byte alignment");
   static_assert(STAGES >= 2, "need at least two stages");
   static_assert(COLS_NEEDED <= 512, "tensor memory overflow");
+  static_assert(HALF % CH == 0 && CH % 16 == 0, "epilogue chunking");
 };
 
 // Instruction descriptor: A K-major (sparse or dense), B K-major, M = 128.
@@ -80,6 +109,21 @@ __host__ __device__ constexpr uint32_t make_idesc() {
   return d;
 }
 
+// Optional timeline trace (compiled in only with NM_TRACE): SM clock-cycle
+// stamps of pipeline events, per CTA (all roles of a CTA share one SM clock).
+#ifdef NM_TRACE
+#define NM_TR(kind, idx)                                                                   \
+  do {                                                                                     \
+    if (a.trace && (idx) < kTraceMax)                                                      \
+      a.trace[(size_t)blockIdx.x * kTraceStride + (kind) * kTraceMax + (idx)] =            \
+          (long long)clock64();                                                            \
+  } while (0)
+#else
+#define NM_TR(kind, idx) \
+  do {                   \
+  } while (0)
+#endif
+
 struct Unit {
   int ct, tt, z, tile, kb0, kb1;
 };
@@ -92,6 +136,45 @@ __device__ __forceinline__ Unit decode_unit(int u, const SpmmArgs& a) {
   w.kb0 = w.z * a.kb_per_split;
   w.kb1 = min(a.n_kb, w.kb0 + a.kb_per_split);
   return w;
+}
+
+// Output element from the 32-bit accumulator: int32; (float)acc * scale; or
+// fp16/bf16 rounded once from the fp32 accumulator (times scale when given).
+template <int OUT>
+__device__ __forceinline__ auto convert_out(uint32_t acc, float s, bool has_scale) {
+  if constexpr (OUT == OUT_I32) {
+    return (int32_t)acc;
+  } else if constexpr (OUT == OUT_F32) {
+    return __fmul_rn(__int2float_rn((int32_t)acc), s);
+  } else {
+    float f = __uint_as_float(acc);
+    if (has_scale) f = __fmul_rn(f, s);
+    if constexpr (OUT == OUT_F16)
+      return __float2half_rn(f);
+    else
+      return __float2bfloat16_rn(f);
+  }
+}
+
+// The units a CTA processes.  Streaming mode: u = blockIdx.x, +gridDim.x, ...
+// X-stationary mode: one contiguous range of tiles in (token tile, channel
+// tile) order, so consecutive tiles share their X tile.
+struct UnitRange {
+  int first, end, step;
+};
+template <bool XS>
+__device__ __forceinline__ UnitRange my_units(const SpmmArgs& a) {
+  UnitRange r;
+  if constexpr (XS) {
+    r.first = (int)(((long long)a.units * blockIdx.x) / gridDim.x);
+    r.end = (int)(((long long)a.units * (blockIdx.x + 1)) / gridDim.x);
+    r.step = 1;
+  } else {
+    r.first = blockIdx.x;
+    r.end = a.units;
+    r.step = gridDim.x;
+  }
+  return r;
 }
 
 template <int OUT>
@@ -119,10 +202,20 @@ __device__ __forceinline__ uint32_t add_acc(uint32_t x, uint32_t y) {
     return __float_as_uint(__uint_as_float(x) + __uint_as_float(y));
 }
 
-template <int DT, int IMG, int BN, int OUT>
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 32)
+    tmem_ld32(taddr, r);
+  else
+    tmem_ld16(taddr, r);
+}
+
+template <int DT, int IMG, int BN, int OUT, int XKB>
 __global__ void __launch_bounds__(kThreads, 1)
-    spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
-  using C = Cfg<DT, IMG, BN>;
+    spmm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                const __grid_constant__ CUtensorMap tmW, const SpmmArgs a) {
+  using C = Cfg<DT, IMG, BN, OUT, XKB>;
+  constexpr bool XS = C::XS;
   constexpr bool SP = C::SP;
   constexpr int KIND = DT == DT_I8 ? 0 : 1;
 
@@ -133,6 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t accf_bar[2];
   __shared__ __align__(8) uint64_t acce_bar[2];
   __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t xfull_bar;   // X-stationary: resident X tile loaded
+  __shared__ __align__(8) uint64_t xempty_bar;  // X-stationary: MMAs reading it have completed
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ int last_sh;
@@ -148,13 +243,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accf_bar[i], 1);
-      mbar_init(&acce_bar[i], 4);
+      mbar_init(&acce_bar[i], kEpiWarps);
     }
     mbar_init(&drain_bar, 1);
+    mbar_init(&xfull_bar, 1);
+    mbar_init(&xempty_bar, 1);
     abort_sh = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&tmX);
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmX);
+    if (a.tma_store) prefetch_tensormap(&tmY);
+    if (a.w_tma) prefetch_tensormap(&tmW);
+  }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
     tmem_relinquish();
@@ -164,6 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   const uint64_t tmo = a.timeout_ns;
+  const UnitRange ur = my_units<XS>(a);
+  uint8_t* const xregion = smem + (size_t)C::STAGES * C::STAGE;  // X-stationary mode only
 
   auto give_up = [&](int code) {
     abort_sh = 1;
@@ -173,25 +276,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int stage = 0, seq = 0;
-      uint32_t phase = 0;
+      int stage = 0, seq = 0, cur_tt = -1;
+      uint32_t phase = 0, xphase = 0;
       uint32_t armed = 0, armed_par = 0;  // per stage: last use carried copies / its parity
+      bool xarmed = false;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
+      for (int u = ur.first; ok && u < ur.end; u += ur.step) {
         const Unit w = decode_unit(u, a);
+        if (XS && w.tt != cur_tt) {
+          // load the X tile of this token tile once the MMAs on the previous one have completed
+          if (!mbar_wait(&xempty_bar, xphase ^ 1u, &abort_sh, tmo)) {
+            give_up(1);
+            break;
+          }
+          mbar_arrive_expect_tx(&xfull_bar, (uint32_t)(a.n_kb * C::B_KBLK));
+          for (int kb = 0; kb < a.n_kb; ++kb) {
+            uint8_t* xs = xregion + (size_t)kb * C::B_KBLK;
+            tma_load_2d(xs, &tmX, &xfull_bar, kb * C::KB, w.tt * BN);
+            tma_load_2d(xs + C::B_BOX, &tmX, &xfull_bar, kb * C::KB + C::KB / 2, w.tt * BN);
+          }
+          xarmed = true;
+          xphase ^= 1u;
+          cur_tt = w.tt;
+        }
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++seq) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
             give_up(1);
             ok = false;
             break;
           }
+          NM_TR(TR_P_ISSUE, seq);
           if (seq != a.inject_skip) {
             uint8_t* st = smem + (size_t)stage * C::STAGE;
             mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)C::STAGE);
-            bulk_load(st, a.bpack + ((size_t)w.ct * a.n_kb + kb) * C::CHUNK, (uint32_t)C::CHUNK,
-                      &full_bar[stage]);
-            tma_load_2d(st + C::CHUNK, &tmX, &full_bar[stage], kb * C::KB, w.tt * BN);
-            tma_load_2d(st + C::CHUNK + C::B_BOX, &tmX, &full_bar[stage], kb * C::KB + C::KB / 2, w.tt * BN);
+            if (a.w_tma)  // the packed image as rows of 128 bytes: one box = one chunk
+              tma_load_2d(st, &tmW, &full_bar[stage], 0, (w.ct * a.n_kb + kb) * (C::CHUNK / 128));
+            else
+              bulk_load(st, a.bpack + ((size_t)w.ct * a.n_kb + kb) * C::CHUNK, (uint32_t)C::CHUNK,
+                        &full_bar[stage]);
+            if constexpr (!XS) {
+              tma_load_2d(st + C::CHUNK, &tmX, &full_bar[stage], kb * C::KB, w.tt * BN);
+              tma_load_2d(st + C::CHUNK + C::B_BOX, &tmX, &full_bar[stage], kb * C::KB + C::KB / 2, w.tt * BN);
+            }
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           } else {
@@ -205,23 +331,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: every copy this thread issued has landed before the CTA exits.
       // Earlier uses of a stage were consumed before it was re-armed, so only
-      // the last armed use of each stage can still be in flight.
+      // the last armed use of each stage (and the last X tile) can still be in flight.
       for (int i = 0; i < C::STAGES; ++i)
         if ((armed >> i) & 1u) mbar_wait(&full_bar[i], (armed_par >> i) & 1u, &abort_sh, tmo);
+      if (xarmed) mbar_wait(&xfull_bar, xphase ^ 1u, &abort_sh, tmo);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc<DT, SP, BN>();
-      int stage = 0, acc = 0, eslot = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int stage = 0, acc = 0, eslot = 0, cur_tt = -1, mseq = 0, mtile = 0;
+      uint32_t phase = 0, acc_phase = 0, xphase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
+      for (int u = ur.first; ok && u < ur.end; u += ur.step) {
         const Unit w = decode_unit(u, a);
+        if (XS && w.tt != cur_tt) {
+          if (cur_tt >= 0) tc_commit(&xempty_bar);  // the old X tile is free once these MMAs finish
+          if (!mbar_wait(&xfull_bar, xphase, &abort_sh, tmo)) {
+            give_up(3);
+            break;
+          }
+          xphase ^= 1u;
+          cur_tt = w.tt;
+        }
         if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &abort_sh, tmo)) {
           give_up(2);
           break;
         }
+        NM_TR(TR_M_ACCE, mtile);
+        ++mtile;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
@@ -230,9 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          NM_TR(TR_M_FULL, mseq);
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + (size_t)stage * C::STAGE);
-          const uint32_t b_addr = a_addr + C::CHUNK;
+          const uint32_t b_addr = XS ? smem_u32(xregion + (size_t)kb * C::B_KBLK) : a_addr + C::CHUNK;
           uint32_t e_tmem = 0;
           if constexpr (SP) {
             e_tmem = tmem + (uint32_t)(C::E_COL0 + eslot * C::E_COLS);
@@ -262,6 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           tc_commit(&empty_bar[stage]);  // frees the smem stage once these MMAs have read it
+          NM_TR(TR_M_DONE, mseq);
+          ++mseq;
           eslot ^= 1;
           if (++stage == C::STAGES) {
             stage = 0;
@@ -281,74 +422,108 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int lg = warp & 3;  // TMEM lane quarter this warp may access
-    const int ep_tid = threadIdx.x - 64;
-    int acc = 0;
+    using OutT = decltype(convert_out<OUT>(0u, 1.0f, false));
+    const int ep_tid = threadIdx.x - 64;  // 0 .. 32*kEpiWarps-1
+    const int ew = warp - 2;              // epilogue warp 0..7
+    const int lq = warp & 3;              // TMEM lane quarter this warp may access
+    const int half = ew >> 2;             // which half of the token columns
+    uint8_t* stage_buf =
+        smem + (size_t)C::STAGES * C::STAGE + C::X_BYTES + (size_t)ew * C::EPI_NB * C::EPI_BUF;
+    int buf = 0, acc = 0;
     uint32_t acc_phase = 0;
-    // One thread waits (bounded) and broadcasts the outcome, so all 128
-    // epilogue threads take the same branch and always meet at the named
-    // barriers; the flag alternates between two slots so a fast thread's next
-    // write cannot overtake a slow thread's read.
+    // One thread waits (bounded) and broadcasts the outcome, so all epilogue
+    // threads take the same branch and always meet at the named barriers; the
+    // flag alternates between two slots so a fast thread's next write cannot
+    // overtake a slow thread's read.
     int iter = 0;
-    for (int u = blockIdx.x; u < a.units; u += gridDim.x, ++iter) {
+    for (int u = ur.first; u < ur.end; u += ur.step, ++iter) {
       const Unit w = decode_unit(u, a);
       if (ep_tid == 0) {
         const bool got = mbar_wait(&accf_bar[acc], acc_phase, &abort_sh, tmo);
         if (!got) give_up(4);
         ep_ok_sh[iter & 1] = got ? 1 : 0;
+        NM_TR(TR_E_START, iter);
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, 32 * kEpiWarps);
       if (!ep_ok_sh[iter & 1]) break;
       tc_fence_after();
-      const int ch = w.ct * kRows + lg * 32 + lane;
+      const int ch0 = w.ct * kRows + lq * 32;  // first channel of this warp's lane quarter
+      const int ch = ch0 + lane;
       const bool ch_ok = ch < a.n_out;
       const bool has_scale = a.scale != nullptr;
       const float s = (has_scale && ch_ok) ? __ldg(a.scale + ch) : 1.0f;
-      const int t0 = w.tt * BN;
-      const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(acc * BN);
+      const int col0 = half * C::HALF;         // first token column of this warp within the tile
+      const int t0 = w.tt * BN + col0;
+      const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(acc * BN + col0);
       if (a.splits == 1) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tbase + 32u * c, r);
+        for (int c = 0; c < C::NCH; ++c) {
+          uint32_t r[C::CH];
+          tmem_ld_n<C::CH>(tbase + (uint32_t)(c * C::CH), r);
           tmem_wait_ld();
+          if (c == C::NCH - 1) {  // all of this warp's columns are in registers: release the accumulator
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce_bar[acc]);
+          }
+          const int tc0 = t0 + c * C::CH;
+          if (a.tma_store) {
+            if (lane == 0) {
+              if (C::EPI_NB == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
+            }
+            __syncwarp();
+            OutT* sb = reinterpret_cast<OutT*>(stage_buf + buf * C::EPI_BUF);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int t = t0 + 32 * c + j;
-            if (ch_ok && t < a.T) store_out<OUT>(a.Y, (size_t)t * a.n_out + ch, r[j], s, has_scale);
+            for (int j = 0; j < C::CH; ++j) sb[j * 32 + lane] = convert_out<OUT>(r[j], s, has_scale);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0 && ch0 < a.n_out && tc0 < a.T) {
+              tma_store_2d(&tmY, sb, ch0, tc0);
+              bulk_commit();
+            }
+            if (C::EPI_NB == 2) buf ^= 1;
+          } else if (ch_ok) {
+            OutT* yp = reinterpret_cast<OutT*>(a.Y) + (size_t)tc0 * a.n_out + ch;
+            const int nvalid = a.T - tc0;
+            if (nvalid >= C::CH) {
+#pragma unroll
+              for (int j = 0; j < C::CH; ++j) yp[(size_t)j * a.n_out] = convert_out<OUT>(r[j], s, has_scale);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::CH; ++j)
+                if (j < nvalid) yp[(size_t)j * a.n_out] = convert_out<OUT>(r[j], s, has_scale);
+            }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acce_bar[acc]);
       } else {
         // split-K: publish this split's partial tile, the last arriving split reduces
         uint32_t* part = reinterpret_cast<uint32_t*>(a.ws);
         const size_t tile_elems = (size_t)BN * kRows;
         uint32_t* mine = part + ((size_t)w.tile * a.splits + w.z) * tile_elems;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tbase + 32u * c, r);
+        for (int c = 0; c < C::NCH; ++c) {
+          uint32_t r[C::CH];
+          tmem_ld_n<C::CH>(tbase + (uint32_t)(c * C::CH), r);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) __stcg(mine + (size_t)(32 * c + j) * kRows + lg * 32 + lane, r[j]);
+          for (int j = 0; j < C::CH; ++j)
+            __stcg(mine + (size_t)(col0 + c * C::CH + j) * kRows + lq * 32 + lane, r[j]);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce_bar[acc]);
         __threadfence();
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 32 * kEpiWarps);
         if (ep_tid == 0) last_sh = (atomicAdd(a.cnt + w.tile, 1) == a.splits - 1);
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 32 * kEpiWarps);
         if (last_sh) {
           __threadfence();
           const uint32_t* tile_base = part + (size_t)w.tile * a.splits * tile_elems;
 #pragma unroll 1
-          for (int col = 0; col < BN; ++col) {
-            const int t = t0 + col;
+          for (int col = col0; col < col0 + C::HALF; ++col) {
+            const int t = w.tt * BN + col;
             if (t >= a.T) break;
-            const size_t off = (size_t)col * kRows + lg * 32 + lane;
+            const size_t off = (size_t)col * kRows + lq * 32 + lane;
             uint32_t sum = __ldcg(tile_base + off);
             for (int z = 1; z < a.splits; ++z) sum = add_acc<DT>(sum, __ldcg(tile_base + z * tile_elems + off));
             if (ch_ok) store_out<OUT>(a.Y, (size_t)t * a.n_out + ch, sum, s, has_scale);
@@ -356,11 +531,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ep_tid == 0) a.cnt[w.tile] = 0;  // re-arm for the next launch
         }
       }
+      if (ep_tid == 0) NM_TR(TR_E_END, iter);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait<0>();  // this warp's tensor stores are complete before the CTA exits
   }
 
   tc_fence_before();
@@ -373,54 +550,55 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ host launch
 
-template <int DT, int IMG, int BN, int OUT>
-static cudaError_t launch_t(const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a, cudaStream_t s) {
-  using C = Cfg<DT, IMG, BN>;
-  auto kern = spmm_kernel<DT, IMG, BN, OUT>;
+template <int DT, int IMG, int BN, int OUT, int XKB>
+static cudaError_t launch_t(const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
+                            const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  using C = Cfg<DT, IMG, BN, OUT, XKB>;
+  auto kern = spmm_kernel<DT, IMG, BN, OUT, XKB>;
   static bool attr_set = false;  // per instantiation; set once per process (single device use)
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<p.grid, kThreads, C::SMEM, s>>>(*tmX, a);
+  kern<<<p.grid, kThreads, C::SMEM, s>>>(*tmX, *tmY, *tmW, a);
   return cudaGetLastError();
 }
 
 template <int DT, int IMG, int OUT>
-static cudaError_t launch_bn(const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+static cudaError_t launch_bn(const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
+                             const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  if (p.xkb > 0) {  // X-stationary mode: INT8, 128-token tiles, up to kXsMaxKb k-blocks (k <= 768)
+    if constexpr (DT == DT_I8) {
+      if (p.bn == 128 && p.xkb <= kXsMaxKb) return launch_t<DT, IMG, 128, OUT, kXsMaxKb>(tmX, tmY, tmW, p, a, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (p.bn) {
-    case 32: return launch_t<DT, IMG, 32, OUT>(tmX, p, a, s);
-    case 64: return launch_t<DT, IMG, 64, OUT>(tmX, p, a, s);
-    case 128: return launch_t<DT, IMG, 128, OUT>(tmX, p, a, s);
+    case 32: return launch_t<DT, IMG, 32, OUT, 0>(tmX, tmY, tmW, p, a, s);
+    case 64: return launch_t<DT, IMG, 64, OUT, 0>(tmX, tmY, tmW, p, a, s);
+    case 128: return launch_t<DT, IMG, 128, OUT, 0>(tmX, tmY, tmW, p, a, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int DT, int OUT>
-static cudaError_t launch_img(int img, const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a, cudaStream_t s) {
-  return img == IMG_SP24 ? launch_bn<DT, IMG_SP24, OUT>(tmX, p, a, s) : launch_bn<DT, IMG_DENSE, OUT>(tmX, p, a, s);
+static cudaError_t launch_img(int img, const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
+                              const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  return img == IMG_SP24 ? launch_bn<DT, IMG_SP24, OUT>(tmX, tmY, tmW, p, a, s)
+                         : launch_bn<DT, IMG_DENSE, OUT>(tmX, tmY, tmW, p, a, s);
 }
 
-cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const Plan& p, const SpmmArgs& a,
-                        cudaStream_t s) {
+cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const CUtensorMap* tmY, const Plan& p,
+                        const SpmmArgs& a, cudaStream_t s) {
+  const CUtensorMap* tmW = &h->tmw;
   switch (h->dt) {
     case DT_I8:
-      return a.scale ? launch_img<DT_I8, OUT_F32>(h->img, tmX, p, a, s)
-                     : launch_img<DT_I8, OUT_I32>(h->img, tmX, p, a, s);
-    case DT_F16: return launch_img<DT_F16, OUT_F16>(h->img, tmX, p, a, s);
-    default: return launch_img<DT_BF16, OUT_BF16>(h->img, tmX, p, a, s);
+      return a.scale ? launch_img<DT_I8, OUT_F32>(h->img, tmX, tmY, tmW, p, a, s)
+                     : launch_img<DT_I8, OUT_I32>(h->img, tmX, tmY, tmW, p, a, s);
+    case DT_F16: return launch_img<DT_F16, OUT_F16>(h->img, tmX, tmY, tmW, p, a, s);
+    default: return launch_img<DT_BF16, OUT_BF16>(h->img, tmX, tmY, tmW, p, a, s);
   }
-}
-
-size_t spmm_smem_bytes(int dt, int img, int bn) {
-  auto pick = [&](auto c) { return (size_t)decltype(c)::SMEM; };
-  if (dt == DT_I8) {
-    if (img == IMG_SP24) return bn == 32 ? pick(Cfg<DT_I8, IMG_SP24, 32>{}) : bn == 64 ? pick(Cfg<DT_I8, IMG_SP24, 64>{}) : pick(Cfg<DT_I8, IMG_SP24, 128>{});
-    return bn == 32 ? pick(Cfg<DT_I8, IMG_DENSE, 32>{}) : bn == 64 ? pick(Cfg<DT_I8, IMG_DENSE, 64>{}) : pick(Cfg<DT_I8, IMG_DENSE, 128>{});
-  }
-  if (img == IMG_SP24) return bn == 32 ? pick(Cfg<DT_F16, IMG_SP24, 32>{}) : bn == 64 ? pick(Cfg<DT_F16, IMG_SP24, 64>{}) : pick(Cfg<DT_F16, IMG_SP24, 128>{});
-  return bn == 32 ? pick(Cfg<DT_F16, IMG_DENSE, 32>{}) : bn == 64 ? pick(Cfg<DT_F16, IMG_DENSE, 64>{}) : pick(Cfg<DT_F16, IMG_DENSE, 128>{});
 }
 
 }  // namespace nm

@@ -58,8 +58,8 @@ def _assert_float_close(Y_gpu: torch.Tensor, Y_ref: np.ndarray, dtype: str):
 
 @pytest.fixture(autouse=True)
 def _no_forced_plan(monkeypatch):
-    monkeypatch.delenv("NMSPMM_FORCE_BN", raising=False)
-    monkeypatch.delenv("NMSPMM_FORCE_SPLITK", raising=False)
+    for k in ("NMSPMM_FORCE_BN", "NMSPMM_FORCE_SPLITK", "NMSPMM_FORCE_XS", "NMSPMM_FORCE_GRID"):
+        monkeypatch.delenv(k, raising=False)
 
 
 # --------------------------------------------------------------------------- compress / decompress
@@ -167,6 +167,36 @@ def test_forced_tiles_and_splits_are_bit_identical(monkeypatch, bn, split):
     for _ in range(2):  # the second call reuses the re-armed split-K counters
         Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
         assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("grid", ["5", "148"])
+@pytest.mark.parametrize("N,M", [(2, 4), (1, 4), (2, 8), (4, 8), (4, 4)])
+@pytest.mark.parametrize("T,n_out,K", [(1000, 300, 768), (129, 200, 512), (640, 384, 256)])
+def test_x_stationary_bit_exact(monkeypatch, grid, N, M, T, n_out, K):
+    """X tile resident across the channel tiles of a CTA's range (token-tile switches included)."""
+    W = _weights("int8", n_out, K, seed=201 + K)
+    X = _acts("int8", T, K, seed=202 + T)
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=203)
+    monkeypatch.setenv("NMSPMM_FORCE_XS", "1")
+    monkeypatch.setenv("NMSPMM_FORCE_GRID", grid)
+    h = nm.nm_compress(W.cuda(), N, M)
+    for scaled in (True, False):
+        Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda() if scaled else None)
+        torch.cuda.synchronize()
+        assert nm.nm_device_status(h) == nm.NM_OK
+        ref = oracle.spmm(X.numpy(), W.numpy(), N, M, scale=s.numpy() if scaled else None)
+        assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("grid", ["3", "11"])
+def test_streaming_mode_many_units_per_cta(monkeypatch, grid):
+    W = _weights("int8", 300, 1024, seed=211)
+    X = _acts("int8", 700, 1024, seed=212)
+    monkeypatch.setenv("NMSPMM_FORCE_XS", "0")
+    monkeypatch.setenv("NMSPMM_FORCE_GRID", grid)
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    Y = nm.nm_spmm(h, X.cuda())
+    assert np.array_equal(Y.cpu().numpy(), oracle.spmm(X.numpy(), W.numpy(), 2, 4))
 
 
 @pytest.mark.parametrize("split", ["1", "4"])
