@@ -76,7 +76,7 @@ EncodeTiledFn encode_fn() {
 // Activation X [T][k] as a 2-D tensor: inner dim k, box = 128 bytes x bn rows,
 // 128-byte swizzle (the layout the MMA's K-major B descriptor expects);
 // out-of-range rows and columns read as zero.
-nm_status make_x_map(nm_handle* h, const void* X, int64_t T, int bn) {
+nm_status make_x_map(nm_handle* h, const void* X, int64_t T, int bn) {  // bn = token rows per box
   if (h->tm_x == X && h->tm_T == T && h->tm_bn == bn) return NM_OK;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
@@ -170,19 +170,55 @@ void out_type(const nm_handle* h, bool scaled, int* es, int* ty) {
 // Split-K: only when even the smallest tile leaves most SMs idle; partials are
 // reduced by the last-arriving CTA, so the reduction costs one extra pass over
 // the tile per split, which is why splits stay bounded by the idle SMs.
-nm::Plan make_plan(const nm_handle* h, int64_t T, int sms) {
+int out_code(const nm_handle* h, bool scaled) {
+  if (h->dt == nm::DT_I8) return scaled ? nm::OUT_F32 : nm::OUT_I32;
+  return h->dt == nm::DT_F16 ? nm::OUT_F16 : nm::OUT_BF16;
+}
+
+nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
   nm::Plan p;
   const int forced_bn = env_int("NMSPMM_FORCE_BN", 0);
   const int forced_split = env_int("NMSPMM_FORCE_SPLITK", 0);
   const int forced_xs = env_int("NMSPMM_FORCE_XS", -1);  // -1 auto, 0 off, 1 on when eligible
   const int forced_grid = env_int("NMSPMM_FORCE_GRID", 0);  // cap on persistent CTAs (tests, sweeps)
   if (forced_grid > 0) sms = std::min(sms, forced_grid);
+  // CTA-pair mode (M = 256 per MMA, one issuing thread per two SMs): whenever
+  // there are enough 256-channel x BN-token tiles to occupy every resident pair.
+  const int forced_pair = env_int("NMSPMM_FORCE_PAIR", -1);  // -1 auto, 0 off, 1 on
+  // Measured on B200: the pair pays off once the k loop is long (k >= 2048), where
+  // per-stage issue cost and X re-reads dominate; shorter k stays on one CTA.
+  const bool pair_default = h->k >= 2048;
+  if ((forced_pair == 1 || (forced_pair == -1 && pair_default)) && forced_split <= 1 && forced_xs != 1) {
+    const int cands[3] = {224, 192, 128};
+    double best_cost = 1e300;
+    for (int bn : cands) {
+      if (forced_bn && bn != forced_bn) continue;
+      int clusters = nm::pair_max_clusters(h->dt, h->img, bn, out_code(h, scaled));
+      if (clusters <= 0) continue;
+      if (forced_grid > 0) clusters = std::min(clusters, std::max(1, forced_grid / 2));
+      const int64_t units = (int64_t)((h->n_ct + 1) / 2) * ((T + bn - 1) / bn);
+      if (forced_pair != 1 && units < clusters) continue;
+      const int64_t rounds = (units + clusters - 1) / clusters;
+      const double cost = (double)rounds * (bn + 48);
+      if (cost < best_cost) {
+        best_cost = cost;
+        p.pair = 1;
+        p.bn = bn;
+        p.n_tt = (int)((T + bn - 1) / bn);
+        p.splits = 1;
+        p.kb_per_split = h->n_kb;
+        p.units = (int)units;
+        p.grid = (int)std::min<int64_t>(units, clusters);
+      }
+    }
+    if (p.pair) return p;
+  }
   // X-stationary mode: INT8 with at most kXsMaxKb k-blocks, several channel tiles
   // sharing each X tile, and enough 128-token tiles to fill the SMs without split-K.
   const int64_t tt128 = (T + 127) / 128;
   const bool xs_ok = h->dt == nm::DT_I8 && h->n_kb <= nm::kXsMaxKb && (forced_bn == 0 || forced_bn == 128) &&
                      forced_split <= 1 && h->n_ct >= 2;
-  if (xs_ok && (forced_xs == 1 || (forced_xs == -1 && tt128 * h->n_ct >= 2 * sms))) {
+  if (xs_ok && forced_xs == 1) {  // measured slower than streaming by default: its write order is scattered
     p.bn = 128;
     p.xkb = h->n_kb;
     p.n_tt = (int)tt128;
@@ -249,8 +285,8 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   if (xs < ys + ybytes && ys < xs + xbytes) return fail(NM_ERR_INVALID, "Y overlaps X");
 
   const int sms = num_sms(h->device);
-  nm::Plan p = make_plan(h, T, sms);
-  st = make_x_map(h, X, T, p.bn);
+  nm::Plan p = make_plan(h, T, sms, scale != nullptr);
+  st = make_x_map(h, X, T, p.pair ? p.bn / 2 : p.bn);
   if (st != NM_OK) return st;
 
   nm::SpmmArgs a{};
@@ -300,7 +336,11 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   }
   int oes, oty;
   out_type(h, scale != nullptr, &oes, &oty);
-  a.tma_store = make_y_map(h, Y, T, oes, oty, std::min(32, p.bn / 2), &st) ? 1 : 0;
+  const int ych = p.pair ? ((p.bn / 2) % 32 == 0 ? 32 : 16) : std::min(32, p.bn / 2);  // epilogue chunk
+  // Direct stores measured faster than staged TMA stores (they keep the TMA unit
+  // for operand loads); the TMA-store epilogue remains selectable.
+  a.tma_store = 0;
+  if (env_int("NMSPMM_TMA_STORE", 0)) a.tma_store = make_y_map(h, Y, T, oes, oty, ych, &st) ? 1 : 0;
   if (st != NM_OK) return st;
   cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "launch SpMM kernel");
@@ -504,8 +544,8 @@ nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y
   const uintptr_t xs = (uintptr_t)X, ys = (uintptr_t)Y;
   if (xs < ys + ybytes && ys < xs + xbytes) return fail(NM_ERR_INVALID, "Y overlaps X");
 
-  const nm::Plan p = make_plan(h, T, num_sms(h->device));
-  st = make_x_map(h, X, T, p.bn);
+  const nm::Plan p = make_plan(h, T, num_sms(h->device), scale != nullptr);
+  st = make_x_map(h, X, T, p.pair ? p.bn / 2 : p.bn);
   if (st != NM_OK) return st;
   nm::SpmmArgs a{};
   a.bpack = h->d_bpack;
@@ -539,7 +579,11 @@ nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y
   }
   int oes, oty;
   out_type(h, scale != nullptr, &oes, &oty);
-  a.tma_store = make_y_map(h, Y, T, oes, oty, std::min(32, p.bn / 2), &st) ? 1 : 0;
+  const int ych = p.pair ? ((p.bn / 2) % 32 == 0 ? 32 : 16) : std::min(32, p.bn / 2);  // epilogue chunk
+  // Direct stores measured faster than staged TMA stores (they keep the TMA unit
+  // for operand loads); the TMA-store epilogue remains selectable.
+  a.tma_store = 0;
+  if (env_int("NMSPMM_TMA_STORE", 0)) a.tma_store = make_y_map(h, Y, T, oes, oty, ych, &st) ? 1 : 0;
   if (st != NM_OK) return st;
   cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch SpMM kernel");

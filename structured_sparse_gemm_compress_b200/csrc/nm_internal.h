@@ -57,6 +57,7 @@ struct Plan {
   int units = 1;      // (tile, split) work units
   int grid = 1;       // persistent CTAs
   int xkb = 0;        // > 0: X-stationary mode holding this many k-blocks of X resident
+  int pair = 0;       // 1: CTA-pair kernel (M = 256 per MMA); grid counts pairs
 };
 
 // Largest number of INT8 k-blocks (256 dense k each) the X-stationary mode keeps resident.
@@ -85,6 +86,8 @@ constexpr int kTraceStride = TR_KINDS * kTraceMax;
 
 cudaError_t launch_compress(const nm_handle* h, const void* W, cudaStream_t s);
 cudaError_t launch_decompress(const nm_handle* h, void* Wout, cudaStream_t s);
+// Resident CTA pairs for the pair kernel of this (dtype, image, token tile, output) or <= 0.
+int pair_max_clusters(int dt, int img, int bn, int out);
 cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const CUtensorMap* tmY, const Plan& p,
                         const SpmmArgs& a, cudaStream_t s);
 

@@ -39,13 +39,15 @@
 
 namespace nm {
 
-enum : int { OUT_I32 = 0, OUT_F32 = 1, OUT_F16 = 2, OUT_BF16 = 3 };
 
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemBudget = 227 * 1024 - 1024;  // dynamic shared memory after 1 KB alignment slack
 
-constexpr int out_bytes(int out) { return (out == OUT_I32 || out == OUT_F32) ? 4 : 2; }
+// OUT template parameter: bits 0-1 = output element (OUT_*), bit 2 = direct-store
+// epilogue (no shared-memory staging, which leaves room for more pipeline stages).
+constexpr int kOutDirect = 4;
+constexpr int out_bytes(int out) { return ((out & 3) == OUT_I32 || (out & 3) == OUT_F32) ? 4 : 2; }
 
 // Kernel configuration.  XKB = 0: streaming mode, every stage carries a packed
 // weight chunk and the matching X boxes.  XKB > 0: X-stationary mode, the
@@ -78,8 +80,9 @@ struct Cfg {
   static constexpr int AVAIL = kSmemBudget - X_BYTES;
   // two staging buffers per warp unless that would leave fewer stages than wanted
   static constexpr int WANT = XS ? 4 : 3;
+  static constexpr bool TS = (OUT & kOutDirect) == 0;   // TMA-store epilogue with staging
   static constexpr int EPI_NB = (AVAIL - 2 * kEpiWarps * EPI_BUF) / STAGE >= WANT ? 2 : 1;
-  static constexpr int EPI_BYTES = EPI_NB * kEpiWarps * EPI_BUF;
+  static constexpr int EPI_BYTES = TS ? EPI_NB * kEpiWarps * EPI_BUF : 0;
   static constexpr int STAGES_FIT = (AVAIL - EPI_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int SMEM = STAGES * STAGE + X_BYTES + EPI_BYTES + 1024;
@@ -90,7 +93,7 @@ struct Cfg {
 };
 
 // Instruction descriptor: A K-major (sparse or dense), B K-major, M = 128.
-template <int DT, bool SP, int BN>
+template <int DT, bool SP, int BN, int M_MMA = 128>
 __host__ __device__ constexpr uint32_t make_idesc() {
   uint32_t d = 0;
   if (SP) d |= 1u << 2;                    // sparse A
@@ -105,7 +108,7 @@ __host__ __device__ constexpr uint32_t make_idesc() {
     d |= f << 10;                          // B
   }
   d |= (uint32_t)(BN >> 3) << 17;          // N
-  d |= (uint32_t)(128 >> 4) << 24;         // M
+  d |= (uint32_t)(M_MMA >> 4) << 24;       // M
   return d;
 }
 
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmX);
-    if (a.tma_store) prefetch_tensormap(&tmY);
+    if (C::TS && a.tma_store) prefetch_tensormap(&tmY);
     if (a.w_tma) prefetch_tensormap(&tmW);
   }
   if (warp == 1) {
@@ -376,15 +379,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (SP) {
             e_tmem = tmem + (uint32_t)(C::E_COL0 + eslot * C::E_COLS);
             const uint32_t e_addr = a_addr + kAtomBytes;
-            tc_cp_128x128b(e_tmem, sdesc_rows16(e_addr));
-            if constexpr (DT == DT_I8) tc_cp_128x128b(e_tmem + 4, sdesc_rows16(e_addr + 2048));
+            if constexpr (DT == DT_I8)
+              tc_cp_128x256b(e_tmem, sdesc_rows16x2(e_addr));
+            else
+              tc_cp_128x128b(e_tmem, sdesc_rows16(e_addr));
           }
+          // descriptors differ only in the start-address field: build once, add offsets
+          const uint64_t ad0 = sdesc_sw128(a_addr), bd0 = sdesc_sw128(b_addr);
 #pragma unroll
           for (int j = 0; j < C::MMAS; ++j) {
             const uint32_t accum = (kb > w.kb0 || j > 0) ? 1u : 0u;
             if constexpr (SP) {
-              const uint64_t ad = sdesc_sw128(a_addr + 32u * j);
-              const uint64_t bd = sdesc_sw128(b_addr + (uint32_t)((j >> 1) * C::B_BOX) + 64u * (j & 1));
+              const uint64_t ad = ad0 + (uint64_t)((32u * j) >> 4);
+              const uint64_t bd = bd0 + (uint64_t)(((uint32_t)((j >> 1) * C::B_BOX) + 64u * (j & 1)) >> 4);
               uint32_t e_addr, id2;
               if constexpr (DT == DT_I8) {
                 e_addr = e_tmem + 2u * j;
@@ -395,8 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               tc_mma_sp<KIND>(d_tmem, ad, bd, e_addr, idesc | id2, accum);
             } else {
-              const uint64_t ad = sdesc_sw128(a_addr + (uint32_t)((j >> 2) * kAtomBytes) + 32u * (j & 3));
-              const uint64_t bd = sdesc_sw128(b_addr + (uint32_t)((j >> 2) * C::B_BOX) + 32u * (j & 3));
+              const uint64_t ad = ad0 + (uint64_t)(((uint32_t)((j >> 2) * kAtomBytes) + 32u * (j & 3)) >> 4);
+              const uint64_t bd = bd0 + (uint64_t)(((uint32_t)((j >> 2) * C::B_BOX) + 32u * (j & 3)) >> 4);
               tc_mma<KIND>(d_tmem, ad, bd, idesc, accum);
             }
           }
@@ -422,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    using OutT = decltype(convert_out<OUT>(0u, 1.0f, false));
+    using OutT = decltype(convert_out<(OUT & 3)>(0u, 1.0f, false));
     const int ep_tid = threadIdx.x - 64;  // 0 .. 32*kEpiWarps-1
     const int ew = warp - 2;              // epilogue warp 0..7
     const int lq = warp & 3;              // TMEM lane quarter this warp may access
@@ -467,14 +474,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&acce_bar[acc]);
           }
           const int tc0 = t0 + c * C::CH;
-          if (a.tma_store) {
+          if (C::TS && a.tma_store) {
             if (lane == 0) {
               if (C::EPI_NB == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
             }
             __syncwarp();
             OutT* sb = reinterpret_cast<OutT*>(stage_buf + buf * C::EPI_BUF);
 #pragma unroll
-            for (int j = 0; j < C::CH; ++j) sb[j * 32 + lane] = convert_out<OUT>(r[j], s, has_scale);
+            for (int j = 0; j < C::CH; ++j) sb[j * 32 + lane] = convert_out<(OUT & 3)>(r[j], s, has_scale);
             fence_async_smem();
             __syncwarp();
             if (lane == 0 && ch0 < a.n_out && tc0 < a.T) {
@@ -487,11 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nvalid = a.T - tc0;
             if (nvalid >= C::CH) {
 #pragma unroll
-              for (int j = 0; j < C::CH; ++j) yp[(size_t)j * a.n_out] = convert_out<OUT>(r[j], s, has_scale);
+              for (int j = 0; j < C::CH; ++j) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
             } else {
 #pragma unroll
               for (int j = 0; j < C::CH; ++j)
-                if (j < nvalid) yp[(size_t)j * a.n_out] = convert_out<OUT>(r[j], s, has_scale);
+                if (j < nvalid) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
             }
           }
         }
@@ -526,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const size_t off = (size_t)col * kRows + lq * 32 + lane;
             uint32_t sum = __ldcg(tile_base + off);
             for (int z = 1; z < a.splits; ++z) sum = add_acc<DT>(sum, __ldcg(tile_base + z * tile_elems + off));
-            if (ch_ok) store_out<OUT>(a.Y, (size_t)t * a.n_out + ch, sum, s, has_scale);
+            if (ch_ok) store_out<(OUT & 3)>(a.Y, (size_t)t * a.n_out + ch, sum, s, has_scale);
           }
           if (ep_tid == 0) a.cnt[w.tile] = 0;  // re-arm for the next launch
         }
@@ -548,6 +555,320 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair kernel
+//
+// Two CTAs on two SMs compute one 256-channel x BN-token tile with
+// tcgen05.mma.cta_group::2 (M = 256: each CTA's 128 rows of the packed weight;
+// N = BN: each CTA holds BN/2 token rows of X).  One thread of the pair leader
+// issues every MMA for both SMs, which halves the per-SM cost of MMA issue, and
+// each SM loads only half of the X tile.  Both CTAs' copies count on the
+// leader's stage barrier; the leader's commits arrive on both CTAs' barriers;
+// the peer's epilogue releases accumulators with remote arrives on the leader.
+// No load uses cluster multicast.
+template <int DT, int IMG, int BN, int OUT>
+struct PairCfg {
+  static constexpr bool SP = IMG == IMG_SP24;
+  static constexpr int KB = kblock_elems(DT);
+  static constexpr int CHUNK = chunk_bytes(DT, IMG);
+  static constexpr int HB = BN / 2;                 // token rows of X held by each CTA
+  static constexpr int B_BOX = HB * 128;
+  static constexpr int STAGE = CHUNK + 2 * B_BOX;
+  static constexpr int MMAS = SP ? 4 : 8;
+  static constexpr int E_COLS = SP ? (DT == DT_I8 ? 8 : 4) : 0;
+  static constexpr int E_COL0 = 2 * BN;
+  static constexpr int COLS_NEEDED = 2 * BN + 2 * E_COLS;
+  static constexpr int TMEM_COLS = COLS_NEEDED <= 256 ? 256 : 512;
+  static constexpr int HALF = BN / 2;               // token columns per epilogue warp
+  static constexpr int CH = (HALF % 32 == 0) ? 32 : 16;
+  static constexpr int NCH = HALF / CH;
+  static constexpr int OES = out_bytes(OUT);
+  static constexpr int EPI_BUF = CH * 32 * OES;
+  static constexpr bool TS = (OUT & kOutDirect) == 0;
+  static constexpr int EPI_NB = (kSmemBudget - 2 * kEpiWarps * EPI_BUF) / STAGE >= 4 ? 2 : 1;
+  static constexpr int EPI_BYTES = TS ? EPI_NB * kEpiWarps * EPI_BUF : 0;
+  static constexpr int STAGES_FIT = (kSmemBudget - EPI_BYTES) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int SMEM = STAGES * STAGE + EPI_BYTES + 1024;
+  static_assert(STAGE % 1024 == 0 && B_BOX % 1024 == 0, "stages keep 1024-byte alignment");
+  static_assert(STAGES >= 2, "need at least two stages");
+  static_assert(COLS_NEEDED <= 512, "tensor memory overflow");
+  static_assert(BN % 32 == 0 && BN <= 256, "pair MMA N");
+  static_assert(HALF % CH == 0, "epilogue chunking");
+};
+
+template <int DT, int IMG, int BN, int OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    spmm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                     const __grid_constant__ CUtensorMap tmW, const SpmmArgs a) {
+  using C = PairCfg<DT, IMG, BN, OUT>;
+  constexpr bool SP = C::SP;
+  constexpr int KIND = DT == DT_I8 ? 0 : 1;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t accf_bar[2];
+  __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+  __shared__ volatile int ep_ok_sh[2];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accf_bar[i], 1);
+      mbar_init(&acce_bar[i], 2 * kEpiWarps);  // both CTAs' epilogue warps release the leader's accumulator
+    }
+    mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmW);
+    if (C::TS && a.tma_store) prefetch_tensormap(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_cg<2>(&tmem_base_sh, C::TMEM_COLS);
+    tmem_relinquish_cg<2>();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA arrive or copy
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint64_t tmo = a.timeout_ns;
+  const uint32_t full_lead0 = mapa_shared(smem_u32(&full_bar[0]), 0);  // leader's stage barriers
+  const uint32_t acce_lead0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
+  const int u_first = (int)cluster_id_x(), u_step = (int)nclusters_x();
+  const int n_pct = (a.n_ct + 1) / 2;  // channel-tile pairs
+
+  auto give_up = [&](int code) {
+    abort_sh = 1;
+    if (a.err) atomicExch(a.err, code);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0, seq = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int u = u_first; ok && u < a.units; u += u_step) {
+        const int pt = u % n_pct, tt = u / n_pct;
+        const int ct = 2 * pt + (int)rank;
+        for (int kb = 0; kb < a.n_kb; ++kb, ++seq) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
+            give_up(1);
+            ok = false;
+            break;
+          }
+          NM_TR(TR_P_ISSUE, seq);
+          if (seq != a.inject_skip) {
+            uint8_t* st = smem + (size_t)stage * C::STAGE;
+            const uint32_t fb = full_lead0 + 8u * (uint32_t)stage;
+            if (leader) mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)(2 * C::STAGE));
+            tma_load_2d_pair(st, &tmW, fb, 0, (ct * a.n_kb + kb) * (C::CHUNK / 128));
+            tma_load_2d_pair(st + C::CHUNK, &tmX, fb, kb * C::KB, tt * BN + (int)rank * C::HB);
+            tma_load_2d_pair(st + C::CHUNK + C::B_BOX, &tmX, fb, kb * C::KB + C::KB / 2,
+                             tt * BN + (int)rank * C::HB);
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          } else {
+            armed &= ~(1u << stage);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: the leader's stage barriers count both CTAs' copies; the peer is
+      // held by the cluster barrier below until the leader has seen them land.
+      if (leader)
+        for (int i = 0; i < C::STAGES; ++i)
+          if ((armed >> i) & 1u) mbar_wait(&full_bar[i], (armed_par >> i) & 1u, &abort_sh, tmo);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = make_idesc<DT, SP, BN, 256>();
+      int stage = 0, acc = 0, eslot = 0, mseq = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int u = u_first; ok && u < a.units; u += u_step) {
+        if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &abort_sh, tmo)) {
+          give_up(2);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < a.n_kb; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_sh, tmo)) {
+            give_up(3);
+            ok = false;
+            break;
+          }
+          NM_TR(TR_M_FULL, mseq);
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + (size_t)stage * C::STAGE);
+          const uint32_t b_addr = a_addr + C::CHUNK;
+          uint32_t e_tmem = 0;
+          if constexpr (SP) {
+            e_tmem = tmem + (uint32_t)(C::E_COL0 + eslot * C::E_COLS);
+            const uint32_t e_addr = a_addr + kAtomBytes;
+            if constexpr (DT == DT_I8)
+              tc_cp_128x256b_pair(e_tmem, sdesc_rows16x2(e_addr));
+            else
+              tc_cp_128x128b_pair(e_tmem, sdesc_rows16(e_addr));
+          }
+          const uint64_t ad0 = sdesc_sw128(a_addr), bd0 = sdesc_sw128(b_addr);
+#pragma unroll
+          for (int j = 0; j < C::MMAS; ++j) {
+            const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+            if constexpr (SP) {
+              const uint64_t ad = ad0 + (uint64_t)((32u * j) >> 4);
+              const uint64_t bd = bd0 + (uint64_t)(((uint32_t)((j >> 1) * C::B_BOX) + 64u * (j & 1)) >> 4);
+              uint32_t e_addr, id2;
+              if constexpr (DT == DT_I8) {
+                e_addr = e_tmem + 2u * j;
+                id2 = 0;
+              } else {
+                e_addr = e_tmem + (uint32_t)(j & ~1);
+                id2 = (uint32_t)(j & 1);
+              }
+              tc_mma_sp_pair<KIND>(d_tmem, ad, bd, e_addr, idesc | id2, accum);
+            } else {
+              const uint64_t ad = ad0 + (uint64_t)(((uint32_t)((j >> 2) * kAtomBytes) + 32u * (j & 3)) >> 4);
+              const uint64_t bd = bd0 + (uint64_t)(((uint32_t)((j >> 2) * C::B_BOX) + 32u * (j & 3)) >> 4);
+              tc_mma_pair<KIND>(d_tmem, ad, bd, idesc, accum);
+            }
+          }
+          tc_commit_pair(&empty_bar[stage], (uint16_t)3);  // frees this stage in both CTAs
+          NM_TR(TR_M_DONE, mseq);
+          ++mseq;
+          eslot ^= 1;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(&accf_bar[acc], (uint16_t)3);  // both CTAs' accumulators are ready
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc_commit_pair(&drain_bar, (uint16_t)3);  // every MMA of this pair has completed
+      mbar_wait(&drain_bar, 0, &abort_sh, tmo);
+    } else if (lane == 0) {
+      mbar_wait(&drain_bar, 0, &abort_sh, tmo);  // peer: the leader's MMAs into this TMEM are done
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    using OutT = decltype(convert_out<(OUT & 3)>(0u, 1.0f, false));
+    const int ep_tid = threadIdx.x - 64;
+    const int ew = warp - 2;
+    const int lq = warp & 3;
+    const int half = ew >> 2;
+    uint8_t* stage_buf = smem + (size_t)C::STAGES * C::STAGE + (size_t)ew * C::EPI_NB * C::EPI_BUF;
+    int buf = 0, acc = 0, iter = 0;
+    uint32_t acc_phase = 0;
+    for (int u = u_first; u < a.units; u += u_step, ++iter) {
+      const int pt = u % n_pct, tt = u / n_pct;
+      const int ct = 2 * pt + (int)rank;
+      if (ep_tid == 0) {
+        const bool got = mbar_wait(&accf_bar[acc], acc_phase, &abort_sh, tmo);
+        if (!got) give_up(4);
+        ep_ok_sh[iter & 1] = got ? 1 : 0;
+        NM_TR(TR_E_START, iter);
+      }
+      named_bar_sync(1, 32 * kEpiWarps);
+      if (!ep_ok_sh[iter & 1]) break;
+      tc_fence_after();
+      const int ch0 = ct * kRows + lq * 32;
+      const int ch = ch0 + lane;
+      const bool ch_ok = ch < a.n_out;
+      const bool has_scale = a.scale != nullptr;
+      const float s = (has_scale && ch_ok) ? __ldg(a.scale + ch) : 1.0f;
+      const int col0 = half * C::HALF;
+      const int t0 = tt * BN + col0;
+      const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(acc * BN + col0);
+#pragma unroll 1
+      for (int c = 0; c < C::NCH; ++c) {
+        uint32_t r[C::CH];
+        tmem_ld_n<C::CH>(tbase + (uint32_t)(c * C::CH), r);
+        tmem_wait_ld();
+        if (c == C::NCH - 1) {  // release the accumulator on the leader
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader)
+              mbar_arrive(&acce_bar[acc]);
+            else
+              mbar_arrive_cluster(acce_lead0 + 8u * (uint32_t)acc);
+          }
+        }
+        const int tc0 = t0 + c * C::CH;
+        if (C::TS && a.tma_store) {
+          if (lane == 0) {
+            if (C::EPI_NB == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
+          }
+          __syncwarp();
+          OutT* sb = reinterpret_cast<OutT*>(stage_buf + buf * C::EPI_BUF);
+#pragma unroll
+          for (int j = 0; j < C::CH; ++j) sb[j * 32 + lane] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0 && ch0 < a.n_out && tc0 < a.T) {
+            tma_store_2d(&tmY, sb, ch0, tc0);
+            bulk_commit();
+          }
+          if (C::EPI_NB == 2) buf ^= 1;
+        } else if (ch_ok) {
+          OutT* yp = reinterpret_cast<OutT*>(a.Y) + (size_t)tc0 * a.n_out + ch;
+          const int nvalid = a.T - tc0;
+          if (nvalid >= C::CH) {
+#pragma unroll
+            for (int j = 0; j < C::CH; ++j) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+          } else {
+#pragma unroll
+            for (int j = 0; j < C::CH; ++j)
+              if (j < nvalid) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+          }
+        }
+      }
+      if (ep_tid == 0) NM_TR(TR_E_END, iter);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  // Teardown: every remote arrive and copy of the pair is done before either
+  // CTA frees tensor memory or exits.
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_cg<2>(tmem, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host launch
 
 template <int DT, int IMG, int BN, int OUT, int XKB>
@@ -565,9 +886,34 @@ static cudaError_t launch_t(const CUtensorMap* tmX, const CUtensorMap* tmY, cons
   return cudaGetLastError();
 }
 
+template <int DT, int IMG, int BN, int OUT>
+static cudaError_t launch_pair_t(const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
+                                 const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  using C = PairCfg<DT, IMG, BN, OUT>;
+  auto kern = spmm_pair_kernel<DT, IMG, BN, OUT>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<2 * p.grid, kThreads, C::SMEM, s>>>(*tmX, *tmY, *tmW, a);  // p.grid = CTA pairs
+  return cudaGetLastError();
+}
+
+int pair_max_clusters(int dt, int img, int bn, int out);
+
 template <int DT, int IMG, int OUT>
 static cudaError_t launch_bn(const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
                              const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  if (p.pair) {
+    switch (p.bn) {
+      case 128: return launch_pair_t<DT, IMG, 128, OUT>(tmX, tmY, tmW, p, a, s);
+      case 192: return launch_pair_t<DT, IMG, 192, OUT>(tmX, tmY, tmW, p, a, s);
+      case 224: return launch_pair_t<DT, IMG, 224, OUT>(tmX, tmY, tmW, p, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   if (p.xkb > 0) {  // X-stationary mode: INT8, 128-token tiles, up to kXsMaxKb k-blocks (k <= 768)
     if constexpr (DT == DT_I8) {
       if (p.bn == 128 && p.xkb <= kXsMaxKb) return launch_t<DT, IMG, 128, OUT, kXsMaxKb>(tmX, tmY, tmW, p, a, s);
@@ -589,16 +935,68 @@ static cudaError_t launch_img(int img, const CUtensorMap* tmX, const CUtensorMap
                          : launch_bn<DT, IMG_DENSE, OUT>(tmX, tmY, tmW, p, a, s);
 }
 
+template <int OUT_TS>
+static cudaError_t launch_dt(const nm_handle* h, const CUtensorMap* tmX, const CUtensorMap* tmY,
+                             const CUtensorMap* tmW, const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  constexpr int D = OUT_TS;  // 0 or kOutDirect
+  switch (h->dt) {
+    case DT_I8:
+      return a.scale ? launch_img<DT_I8, OUT_F32 | D>(h->img, tmX, tmY, tmW, p, a, s)
+                     : launch_img<DT_I8, OUT_I32 | D>(h->img, tmX, tmY, tmW, p, a, s);
+    case DT_F16: return launch_img<DT_F16, OUT_F16 | D>(h->img, tmX, tmY, tmW, p, a, s);
+    default: return launch_img<DT_BF16, OUT_BF16 | D>(h->img, tmX, tmY, tmW, p, a, s);
+  }
+}
+
 cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const CUtensorMap* tmY, const Plan& p,
                         const SpmmArgs& a, cudaStream_t s) {
   const CUtensorMap* tmW = &h->tmw;
-  switch (h->dt) {
-    case DT_I8:
-      return a.scale ? launch_img<DT_I8, OUT_F32>(h->img, tmX, tmY, tmW, p, a, s)
-                     : launch_img<DT_I8, OUT_I32>(h->img, tmX, tmY, tmW, p, a, s);
-    case DT_F16: return launch_img<DT_F16, OUT_F16>(h->img, tmX, tmY, tmW, p, a, s);
-    default: return launch_img<DT_BF16, OUT_BF16>(h->img, tmX, tmY, tmW, p, a, s);
+  return a.tma_store ? launch_dt<0>(h, tmX, tmY, tmW, p, a, s) : launch_dt<kOutDirect>(h, tmX, tmY, tmW, p, a, s);
+}
+
+// Pairs that can be resident at once for a pair-kernel configuration (cached).
+template <int DT, int IMG, int BN, int OUT>
+static int max_clusters_t() {
+  static int cached = 0;
+  if (!cached) {
+    using C = PairCfg<DT, IMG, BN, OUT>;
+    auto kern = spmm_pair_kernel<DT, IMG, BN, OUT>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.attrs = nullptr;  // the kernel declares its cluster shape (2 CTAs) at compile time
+    cfg.numAttrs = 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cached = n > 0 ? n : -1;
   }
+  return cached;
+}
+
+int pair_max_clusters(int dt, int img, int bn, int out) {
+  // All configurations share threads and (nearly) shared memory: one query per dtype/bn suffices.
+  int n = -1;
+  if (dt == DT_I8) {
+    const bool f32 = out == OUT_F32;
+    if (img == IMG_SP24) n = bn == 224 ? (f32 ? max_clusters_t<DT_I8, IMG_SP24, 224, OUT_F32>() : max_clusters_t<DT_I8, IMG_SP24, 224, OUT_I32>())
+                       : bn == 192 ? (f32 ? max_clusters_t<DT_I8, IMG_SP24, 192, OUT_F32>() : max_clusters_t<DT_I8, IMG_SP24, 192, OUT_I32>())
+                                   : (f32 ? max_clusters_t<DT_I8, IMG_SP24, 128, OUT_F32>() : max_clusters_t<DT_I8, IMG_SP24, 128, OUT_I32>());
+    else n = bn == 224 ? (f32 ? max_clusters_t<DT_I8, IMG_DENSE, 224, OUT_F32>() : max_clusters_t<DT_I8, IMG_DENSE, 224, OUT_I32>())
+           : bn == 192 ? (f32 ? max_clusters_t<DT_I8, IMG_DENSE, 192, OUT_F32>() : max_clusters_t<DT_I8, IMG_DENSE, 192, OUT_I32>())
+                       : (f32 ? max_clusters_t<DT_I8, IMG_DENSE, 128, OUT_F32>() : max_clusters_t<DT_I8, IMG_DENSE, 128, OUT_I32>());
+  } else if (dt == DT_F16) {
+    n = img == IMG_SP24 ? (bn == 224 ? max_clusters_t<DT_F16, IMG_SP24, 224, OUT_F16>() : bn == 192 ? max_clusters_t<DT_F16, IMG_SP24, 192, OUT_F16>() : max_clusters_t<DT_F16, IMG_SP24, 128, OUT_F16>())
+                        : (bn == 224 ? max_clusters_t<DT_F16, IMG_DENSE, 224, OUT_F16>() : bn == 192 ? max_clusters_t<DT_F16, IMG_DENSE, 192, OUT_F16>() : max_clusters_t<DT_F16, IMG_DENSE, 128, OUT_F16>());
+  } else {
+    n = img == IMG_SP24 ? (bn == 224 ? max_clusters_t<DT_BF16, IMG_SP24, 224, OUT_BF16>() : bn == 192 ? max_clusters_t<DT_BF16, IMG_SP24, 192, OUT_BF16>() : max_clusters_t<DT_BF16, IMG_SP24, 128, OUT_BF16>())
+                        : (bn == 224 ? max_clusters_t<DT_BF16, IMG_DENSE, 224, OUT_BF16>() : bn == 192 ? max_clusters_t<DT_BF16, IMG_DENSE, 192, OUT_BF16>() : max_clusters_t<DT_BF16, IMG_DENSE, 128, OUT_BF16>());
+  }
+  return n;
 }
 
 }  // namespace nm

@@ -58,7 +58,8 @@ def _assert_float_close(Y_gpu: torch.Tensor, Y_ref: np.ndarray, dtype: str):
 
 @pytest.fixture(autouse=True)
 def _no_forced_plan(monkeypatch):
-    for k in ("NMSPMM_FORCE_BN", "NMSPMM_FORCE_SPLITK", "NMSPMM_FORCE_XS", "NMSPMM_FORCE_GRID"):
+    for k in ("NMSPMM_FORCE_BN", "NMSPMM_FORCE_SPLITK", "NMSPMM_FORCE_XS", "NMSPMM_FORCE_GRID",
+              "NMSPMM_FORCE_PAIR", "NMSPMM_TMA_STORE"):
         monkeypatch.delenv(k, raising=False)
 
 
@@ -116,7 +117,9 @@ def test_hand_examples_on_gpu():
 @pytest.mark.parametrize("N,M", PATTERNS)
 @pytest.mark.parametrize("scaled", [False, True])
 @pytest.mark.parametrize("T,n_out,K", [(300, 200, 784), (1, 128, 256), (197, 96, 96), (64, 384, 3072)])
-def test_spmm_int8_bit_exact(N, M, scaled, T, n_out, K):
+@pytest.mark.parametrize("tma_store", ["0", "1"])
+def test_spmm_int8_bit_exact(monkeypatch, N, M, scaled, T, n_out, K, tma_store):
+    monkeypatch.setenv("NMSPMM_TMA_STORE", tma_store)
     W = _weights("int8", n_out, K, seed=7 + K)
     X = _acts("int8", T, K, seed=8 + T)
     s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=9) if scaled else None
@@ -134,7 +137,9 @@ def test_spmm_int8_bit_exact(N, M, scaled, T, n_out, K):
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("N,M", PATTERNS)
 @pytest.mark.parametrize("T,n_out,K", [(300, 200, 392), (5, 256, 1024), (131, 64, 4096)])
-def test_spmm_float_within_tolerance(dtype, N, M, T, n_out, K):
+@pytest.mark.parametrize("tma_store", ["0", "1"])
+def test_spmm_float_within_tolerance(monkeypatch, dtype, N, M, T, n_out, K, tma_store):
+    monkeypatch.setenv("NMSPMM_TMA_STORE", tma_store)
     W = _weights(dtype, n_out, K, seed=17 + K)
     X = _acts(dtype, T, K, seed=18 + T)
     h = nm.nm_compress(W.cuda(), N, M)
@@ -172,12 +177,15 @@ def test_forced_tiles_and_splits_are_bit_identical(monkeypatch, bn, split):
 @pytest.mark.parametrize("grid", ["5", "148"])
 @pytest.mark.parametrize("N,M", [(2, 4), (1, 4), (2, 8), (4, 8), (4, 4)])
 @pytest.mark.parametrize("T,n_out,K", [(1000, 300, 768), (129, 200, 512), (640, 384, 256)])
-def test_x_stationary_bit_exact(monkeypatch, grid, N, M, T, n_out, K):
+@pytest.mark.parametrize("tma_store", ["0", "1"])
+def test_x_stationary_bit_exact(monkeypatch, grid, N, M, T, n_out, K, tma_store):
     """X tile resident across the channel tiles of a CTA's range (token-tile switches included)."""
+    monkeypatch.setenv("NMSPMM_TMA_STORE", tma_store)
     W = _weights("int8", n_out, K, seed=201 + K)
     X = _acts("int8", T, K, seed=202 + T)
     s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=203)
     monkeypatch.setenv("NMSPMM_FORCE_XS", "1")
+    monkeypatch.setenv("NMSPMM_FORCE_PAIR", "0")
     monkeypatch.setenv("NMSPMM_FORCE_GRID", grid)
     h = nm.nm_compress(W.cuda(), N, M)
     for scaled in (True, False):
@@ -188,11 +196,50 @@ def test_x_stationary_bit_exact(monkeypatch, grid, N, M, T, n_out, K):
         assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
 
 
+@pytest.mark.parametrize("bn", ["128", "192", "224"])
+@pytest.mark.parametrize("grid", ["6", "148"])
+@pytest.mark.parametrize("N,M", [(2, 4), (1, 4), (2, 8), (4, 8), (8, 8)])
+@pytest.mark.parametrize("T,n_out,K", [(1000, 300, 768), (130, 640, 512), (450, 256, 1280)])
+@pytest.mark.parametrize("tma_store", ["0", "1"])
+def test_cta_pair_bit_exact(monkeypatch, bn, grid, N, M, T, n_out, K, tma_store):
+    """CTA-pair kernel: ragged T, odd channel-tile counts (n_out=300), several tiles per pair."""
+    monkeypatch.setenv("NMSPMM_TMA_STORE", tma_store)
+    W = _weights("int8", n_out, K, seed=301 + K)
+    X = _acts("int8", T, K, seed=302 + T)
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=303)
+    monkeypatch.setenv("NMSPMM_FORCE_PAIR", "1")
+    monkeypatch.setenv("NMSPMM_FORCE_BN", bn)
+    monkeypatch.setenv("NMSPMM_FORCE_GRID", grid)
+    h = nm.nm_compress(W.cuda(), N, M)
+    for scaled in (True, False):
+        Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda() if scaled else None)
+        torch.cuda.synchronize()
+        assert nm.nm_device_status(h) == nm.NM_OK
+        ref = oracle.spmm(X.numpy(), W.numpy(), N, M, scale=s.numpy() if scaled else None)
+        assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("bn", ["128", "224"])
+@pytest.mark.parametrize("N,M", [(2, 4), (2, 8), (4, 8)])
+def test_cta_pair_float_within_tolerance(monkeypatch, dtype, bn, N, M):
+    W = _weights(dtype, 384, 1024, seed=311)
+    X = _acts(dtype, 500, 1024, seed=312)
+    monkeypatch.setenv("NMSPMM_FORCE_PAIR", "1")
+    monkeypatch.setenv("NMSPMM_FORCE_BN", bn)
+    h = nm.nm_compress(W.cuda(), N, M)
+    Y = nm.nm_spmm(h, X.cuda())
+    torch.cuda.synchronize()
+    assert nm.nm_device_status(h) == nm.NM_OK
+    _assert_float_close(Y, oracle.spmm(_np(X, dtype), _np(W, dtype), N, M, dtype=dtype), dtype)
+
+
 @pytest.mark.parametrize("grid", ["3", "11"])
 def test_streaming_mode_many_units_per_cta(monkeypatch, grid):
     W = _weights("int8", 300, 1024, seed=211)
     X = _acts("int8", 700, 1024, seed=212)
     monkeypatch.setenv("NMSPMM_FORCE_XS", "0")
+    monkeypatch.setenv("NMSPMM_FORCE_PAIR", "0")
     monkeypatch.setenv("NMSPMM_FORCE_GRID", grid)
     h = nm.nm_compress(W.cuda(), 2, 4)
     Y = nm.nm_spmm(h, X.cuda())
