@@ -209,6 +209,136 @@ def run_reference(args, rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------- other workloads
+
+
+def roofline_point(l, us: float, pk: dict) -> dict:
+    """Roofline of one problem: t = max(ops / tensor peak, bytes / HBM peak).
+
+    Tensor peaks derive from the measured bf16 dense peak with NVIDIA's nominal
+    ratios: INT8 dense = 2 x bf16, FP16/BF16 dense = bf16, 2:4-sparse = 2 x dense
+    (1:4, 2:4, 2:8 run on the sparse pipe; 4:8 and N = M on the dense pipe)."""
+    dense_peak = pk["bf16_tflops"] * (2.0 if l.dtype == inputs.INT8 else 1.0)
+    sparse = (l.N, l.M) in ((1, 4), (2, 4), (2, 8))
+    tc_peak = dense_peak * (2.0 if sparse else 1.0)
+    ops = l.dense_ops()
+    t_tc = ops / (tc_peak * 1e12) * 1e6
+    bytes_ = alg_bytes_any(l)
+    t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9) * 1e6
+    t_roof = max(t_tc, t_hbm)
+    return {"us": round(us, 2), "dense_eq_tops": round(ops / us / 1e6, 1),
+            "bound": "tensor" if t_tc > t_hbm else "hbm", "roofline_us": round(t_roof, 2),
+            "frac": round(t_roof / us, 3)}
+
+
+def alg_bytes_any(l) -> int:
+    """Algorithmic bytes of one SpMM launch for any dtype/output."""
+    import math
+    es = 1 if l.dtype == inputs.INT8 else 2
+    kept = l.n_out * (l.K // l.M) * l.N
+    wbytes = (kept * es + (kept * math.ceil(math.log2(l.M)) + 7) // 8) if l.N != l.M else l.n_out * l.K * es
+    out_es = (4 if l.dtype == inputs.INT8 else 2)
+    return l.T * l.K * es + wbytes + l.T * l.n_out * out_es + (4 * l.n_out if l.scaled else 0)
+
+
+def run_config(name: str, args) -> None:
+    import structured_sparse_gemm_compress_b200 as nm
+
+    torch.cuda.set_device(0)
+    pk = peaks()
+    if name == "single":
+        ls, desc = inputs.single_layer(), "single ViT-B linear, INT8 2:4, T=197, 768->768, int32 out"
+    elif name == "vitl":
+        ls, desc = inputs.vit_l_fp16(), "ViT-L/16 linears, batch 32 (T=6304), FP16, N:M in {1:4,2:4,2:8}"
+    elif name == "swin":
+        ls, desc = inputs.swin_t_int8(), "Swin-T linears per stage, batch 128, INT8 + scale, N:M in {2:4,2:8}"
+    elif name in ("mixed1", "mixed256"):
+        T = 197 if name == "mixed1" else 50432
+        ls, desc = inputs.vit_b_mixed(T), f"all 48 ViT-B linears at T={T}, per-layer N:M from {{dense,4:8,2:4,2:8,1:4}}"
+    else:
+        raise SystemExit(f"unknown config {name}")
+    stream = torch.cuda.current_stream()
+    probs = []
+    for l in ls:
+        W, X, sc = l.weight().cuda(), l.activation().cuda(), l.scale()
+        sc = None if sc is None else sc.cuda()
+        h = nm.nm_compress(W, l.N, l.M)
+        Y = torch.empty((l.T, l.n_out), dtype=nm.out_dtype(h, sc is not None), device="cuda")
+        probs.append((l, W, X, sc, h, Y))
+    torch.cuda.synchronize()
+
+    def run_all(evs=None):
+        for i, (l, W, X, sc, h, Y) in enumerate(probs):
+            if evs is not None:
+                evs[i][0].record(stream)
+            nm.nm_spmm(h, X, Y=Y, scale=sc, stream=stream)
+            if evs is not None:
+                evs[i][1].record(stream)
+
+    reps = max(3, args.steps)
+    for _ in range(args.warmup):
+        run_all()
+    torch.cuda.synchronize()
+    # the sequence back to back in one stream, captured as one CUDA graph
+    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in probs]
+           for _ in range(reps)]
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+        for r in range(reps):
+            for i, (l, W, X, sc, h, Y) in enumerate(probs):
+                evs[r][i][0].record(cap)
+                nm.nm_spmm(h, X, Y=Y, scale=sc, stream=cap)
+                evs[r][i][1].record(cap)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    seq_ms = a.elapsed_time(b) / reps
+    for h in (p[4] for p in probs):
+        if nm.nm_device_status(h) != nm.NM_OK:
+            raise RuntimeError(nm.nm_last_error())
+    per = []
+    for i, (l, W, X, sc, h, Y) in enumerate(probs):
+        us = statistics.median(evs[r][i][0].elapsed_time(evs[r][i][1]) * 1e3 for r in range(reps))
+        rp = roofline_point(l, us, pk)
+        # same-shape cuBLAS dense GEMM through torch (context)
+        if l.dtype == inputs.INT8 and l.T > 16:
+            fn = (lambda X=X, W=W: torch._int_mm(X, W.t()))
+        elif l.dtype != inputs.INT8:
+            fn = (lambda X=X, W=W: torch.matmul(X, W.t()))
+        else:
+            fn = None
+        if fn is not None:
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(10):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            rp["cublas_dense_us"] = round(e0.elapsed_time(e1) * 100, 2)
+        rp["problem"] = f"{l.name}/{l.nm}"
+        rp["T,K,n_out"] = [l.T, l.K, l.n_out]
+        per.append(rp)
+    total_ops = sum(l.dense_ops() for l in ls)
+    tot_roof = sum(p["roofline_us"] for p in per)
+    sum_us = sum(p["us"] for p in per)
+    line = {"config": {"workload": desc}, "metric": "dense-equivalent TOPS over the sequence", "unit": "TOPS",
+            "value": total_ops / (seq_ms * 1e-3) / 1e12, "sequence_us": round(seq_ms * 1e3, 2),
+            "sum_of_kernel_us": round(sum_us, 2), "roofline_us": round(tot_roof, 2),
+            "roofline_frac": round(tot_roof / (seq_ms * 1e3), 3), "dtype": ls[0].dtype, "data": "synthetic",
+            "launch": "CUDA graph of the sequence", "reps": reps, "per_problem": per}
+    if any("cublas_dense_us" in p for p in per):
+        line["cublas_dense_sum_us"] = round(sum(p.get("cublas_dense_us", 0.0) for p in per), 2)
+    print(json.dumps(line), flush=True)
+
+
 # --------------------------------------------------------------------------- GPU arm
 
 
@@ -222,6 +352,8 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
+    ap.add_argument("--config", default=None, choices=["single", "vitl", "swin", "mixed1", "mixed256"],
+                    help="measure another workload (one JSON line) instead of the default ViT-B INT8 set")
     ap.add_argument("--only", action="append", default=[],
                     help="restrict to problems like vitb.fc1/2:4 (profiling a single kernel shape)")
     args = ap.parse_args()
@@ -232,6 +364,10 @@ def main() -> None:
     world, rank, local_rank = rank_env()
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.config is not None:
+        if rank == 0:
+            run_config(args.config, args)
         return
 
     import structured_sparse_gemm_compress_b200 as nm

@@ -185,9 +185,9 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
   // CTA-pair mode (M = 256 per MMA, one issuing thread per two SMs): whenever
   // there are enough 256-channel x BN-token tiles to occupy every resident pair.
   const int forced_pair = env_int("NMSPMM_FORCE_PAIR", -1);  // -1 auto, 0 off, 1 on
-  // Measured on B200: the pair pays off once the k loop is long (k >= 2048), where
+  // Measured on B200: the pair pays off once the k loop is long (>= 2 KB of X per token), where
   // per-stage issue cost and X re-reads dominate; shorter k stays on one CTA.
-  const bool pair_default = h->k >= 2048;
+  const bool pair_default = h->k * nm::elem_bytes(h->dt) >= 2048;  // >= 2 KB of X per token
   if ((forced_pair == 1 || (forced_pair == -1 && pair_default)) && forced_split <= 1 && forced_xs != 1) {
     const int cands[3] = {224, 192, 128};
     double best_cost = 1e300;

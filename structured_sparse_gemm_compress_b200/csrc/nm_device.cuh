@@ -142,6 +142,16 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 
+// --- programmatic dependent launch
+// Let the next kernel of the stream start its prologue once every CTA of this
+// grid has issued this (or exited).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the previous kernel of the stream has completed and its memory
+// operations are visible (returns at once when there is none).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // --- thread-block clusters (CTA pairs)
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -266,6 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Prologue done: the next kernel may start its own; global memory is touched
+  // only after the previous kernel has completed (RAW/WAW order across launches).
+  pdl_launch_dependents();
+  pdl_wait();
   const uint32_t tmem = tmem_base_sh;
   const uint64_t tmo = a.timeout_ns;
   const UnitRange ur = my_units<XS>(a);
@@ -526,14 +530,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last_sh) {
           __threadfence();
           const uint32_t* tile_base = part + (size_t)w.tile * a.splits * tile_elems;
+          // eight columns at a time, every split's loads in flight before any add
+          constexpr int RC = C::HALF < 8 ? C::HALF : 8;
 #pragma unroll 1
-          for (int col = col0; col < col0 + C::HALF; ++col) {
-            const int t = w.tt * BN + col;
-            if (t >= a.T) break;
-            const size_t off = (size_t)col * kRows + lq * 32 + lane;
-            uint32_t sum = __ldcg(tile_base + off);
-            for (int z = 1; z < a.splits; ++z) sum = add_acc<DT>(sum, __ldcg(tile_base + z * tile_elems + off));
-            if (ch_ok) store_out<(OUT & 3)>(a.Y, (size_t)t * a.n_out + ch, sum, s, has_scale);
+          for (int cb = col0; cb < col0 + C::HALF; cb += RC) {
+            uint32_t sum[RC];
+            const uint32_t* src = tile_base + (size_t)cb * kRows + lq * 32 + lane;
+#pragma unroll
+            for (int q = 0; q < RC; ++q) sum[q] = __ldcg(src + (size_t)q * kRows);
+            for (int z = 1; z < a.splits; ++z) {
+              uint32_t v[RC];
+#pragma unroll
+              for (int q = 0; q < RC; ++q) v[q] = __ldcg(src + z * tile_elems + (size_t)q * kRows);
+#pragma unroll
+              for (int q = 0; q < RC; ++q) sum[q] = add_acc<DT>(sum[q], v[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < RC; ++q) {
+              const int t = w.tt * BN + cb + q;
+              if (ch_ok && t < a.T) store_out<(OUT & 3)>(a.Y, (size_t)t * a.n_out + ch, sum[q], s, has_scale);
+            }
           }
           if (ep_tid == 0) a.cnt[w.tile] = 0;  // re-arm for the next launch
         }
@@ -645,6 +661,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA arrive or copy
   tc_fence_after();
+  pdl_launch_dependents();
+  pdl_wait();
   const uint32_t tmem = tmem_base_sh;
   const uint64_t tmo = a.timeout_ns;
   const uint32_t full_lead0 = mapa_shared(smem_u32(&full_bar[0]), 0);  // leader's stage barriers
@@ -871,6 +889,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ host launch
 
+// Launch with programmatic stream serialization, so the kernel's prologue can
+// overlap the tail of the previous kernel in the stream (see pdl_wait).
+template <typename Kern>
+static cudaError_t launch_pdl(Kern kern, dim3 grid, int smem, cudaStream_t s, const CUtensorMap& tmX,
+                              const CUtensorMap& tmY, const CUtensorMap& tmW, const SpmmArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmX, tmY, tmW, a);
+}
+
 template <int DT, int IMG, int BN, int OUT, int XKB>
 static cudaError_t launch_t(const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
                             const Plan& p, const SpmmArgs& a, cudaStream_t s) {
@@ -882,8 +918,7 @@ static cudaError_t launch_t(const CUtensorMap* tmX, const CUtensorMap* tmY, cons
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<p.grid, kThreads, C::SMEM, s>>>(*tmX, *tmY, *tmW, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(p.grid), C::SMEM, s, *tmX, *tmY, *tmW, a);
 }
 
 template <int DT, int IMG, int BN, int OUT>
@@ -897,8 +932,7 @@ static cudaError_t launch_pair_t(const CUtensorMap* tmX, const CUtensorMap* tmY,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<2 * p.grid, kThreads, C::SMEM, s>>>(*tmX, *tmY, *tmW, a);  // p.grid = CTA pairs
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(2 * p.grid), C::SMEM, s, *tmX, *tmY, *tmW, a);  // p.grid = CTA pairs
 }
 
 int pair_max_clusters(int dt, int img, int bn, int out);
