@@ -60,6 +60,10 @@ def _load():
         lib.oracle_gemm_f16.argtypes = [p, i64, i64, p, i64, i32, p, p]
         lib.oracle_idx_pitch.argtypes = [i64, i32, i32]
         lib.oracle_idx_pitch.restype = i64
+        lib.oracle_epilogue_i8.argtypes = [p, i64, i64, p, p, i32, ctypes.c_float, p, p, p]
+        lib.oracle_epilogue_f.argtypes = [p, i64, i64, p, p, i32, p]
+        lib.oracle_gelu.argtypes = [ctypes.c_double]
+        lib.oracle_gelu.restype = ctypes.c_double
         lib.oracle_threads.restype = i32
         lib.oracle_set_threads.argtypes = [i32]
         _lib = lib
@@ -162,3 +166,81 @@ def spmm(X: np.ndarray, W: np.ndarray, N: int, M: int, scale: np.ndarray | None 
     values, idx = compress(W, N, M, dtype)
     Wm = decompress(values, idx, W.shape[0], W.shape[1], N, M, dtype)
     return gemm(X, Wm, scale, dtype)
+
+
+ACTS = {"none": 0, "gelu": 1}
+OUTS = ("float32", "float16", "bfloat16", "int8")
+
+
+def gelu(x: float) -> float:
+    """The erf form of GELU, x/2 * (1 + erf(x / sqrt 2)), in fp64."""
+    return float(_load().oracle_gelu(float(x)))
+
+
+def epilogue(acc: np.ndarray, scale: np.ndarray | None = None, bias: np.ndarray | None = None,
+             act: str = "none", out: str = "float32", out_scale: float = 1.0) -> dict:
+    """The fused output stage on a GEMM accumulator [T, n_out].
+
+    ``acc`` int32 (INT8 path) or float64 (FP16/BF16 path, the fp64 sum).
+    Returns a dict with
+      ``pre``   -- float64 value after scale, bias and activation;
+      ``exact`` -- the output tensor the kernel must reproduce bit for bit,
+                   or None where several results are correct (GELU: the
+                   kernel evaluates erf in fp32; FP16/BF16 inputs: any
+                   summation order);
+      ``q``     -- for ``out='int8'``: the int8 codes decided from ``pre``
+                   (exact when ``exact`` is not None);
+      ``q_pre`` -- for ``out='int8'``: the value that was rounded (fp64).
+    Rounding to float16 uses numpy's float32 -> float16 conversion and to
+    bfloat16 torch's, both round-to-nearest-even, applied to the exact fp32
+    result of the INT8 path.
+    """
+    if act not in ACTS or out not in OUTS:
+        raise ValueError("bad act/out")
+    acc = np.ascontiguousarray(acc)
+    T, n_out = acc.shape
+    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.float32)
+    bi = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    lib = _load()
+    pre = np.zeros((T, n_out), dtype=np.float64)
+    res = {"pre": pre, "exact": None}
+    if acc.dtype == np.int32:
+        v32 = np.zeros((T, n_out), dtype=np.float32)
+        q = np.zeros((T, n_out), dtype=np.int8)
+        rc = lib.oracle_epilogue_i8(_ptr(acc), T, n_out, None if sc is None else _ptr(sc),
+                                    None if bi is None else _ptr(bi), ACTS[act], float(out_scale),
+                                    _ptr(pre), _ptr(v32), _ptr(q))
+        if rc != 0:
+            raise ValueError(f"oracle_epilogue_i8 failed (rc={rc})")
+        if out == "int8":
+            res["q"] = q
+            res["q_pre"] = pre * np.float64(np.float32(out_scale)) if act == "gelu" else \
+                (v32 * np.float32(out_scale)).astype(np.float64)
+            if act == "none":
+                res["exact"] = q
+        elif act == "none":
+            if out == "float32":
+                res["exact"] = v32
+            elif out == "float16":
+                res["exact"] = v32.astype(np.float16)
+            else:
+                import torch
+                res["exact"] = torch.from_numpy(v32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        return res
+    if acc.dtype != np.float64 or out == "int8":
+        raise ValueError("float path: float64 accumulator, float output")
+    rc = lib.oracle_epilogue_f(_ptr(acc), T, n_out, None if sc is None else _ptr(sc),
+                               None if bi is None else _ptr(bi), ACTS[act], _ptr(pre))
+    if rc != 0:
+        raise ValueError(f"oracle_epilogue_f failed (rc={rc})")
+    return res
+
+
+def spmm_epilogue(X: np.ndarray, W: np.ndarray, N: int, M: int, scale=None, bias=None, act="none",
+                  out="float32", out_scale=1.0, dtype: str | None = None) -> dict:
+    """The whole path with the fused output stage: compress, decompress, the
+    raw GEMM accumulator (int32 or fp64), then ``epilogue``."""
+    values, idx = compress(W, N, M, dtype)
+    Wm = decompress(values, idx, W.shape[0], W.shape[1], N, M, dtype)
+    acc = gemm(X, Wm, None, dtype)
+    return epilogue(acc, scale, bias, act, out, out_scale)

@@ -24,9 +24,15 @@
  *     (build with -ffp-contract=off);
  *   - FP16/BF16 GEMM: inputs decoded exactly to double, fp64 accumulation,
  *     result returned in fp64.
+ *   - fused output stage (per-channel scale, per-channel bias, GELU, int8
+ *     requantisation): the library's own definition, see oracle_epilogue_i8;
+ *     the paper does not discuss the output stage.
  *
  * Parity pins (tests/test_oracle.py): hand-worked 4x8 examples, brute-force
- * subset enumeration, invariants, and exact integer matmul cross-checks.
+ * subset enumeration, invariants, and exact integer matmul cross-checks; for
+ * the output stage, hand-worked rounding/saturation cases
+ * (tests/golden/epilogue_hand.json), the standard normal CDF table for GELU
+ * and the identity GELU(x) - GELU(-x) = x.
  */
 #include <math.h>
 #include <stdint.h>
@@ -216,3 +222,76 @@ int oracle_gemm_f16(const uint16_t *X, int64_t T, int64_t K, const uint16_t *Wm,
     }
     return 0;
 }
+
+/*
+ * Fused output stage applied to the GEMM accumulator.  The paper does not
+ * discuss the output stage (its kernel description ends at the MMA), so this
+ * is the library's own definition, written out step by step:
+ *
+ *   v = a                              a = (float)acc, rounded to nearest
+ *   v = v * scale[n]   (if scale)      one rounded fp32 multiply
+ *   v = v + bias[n]    (if bias)       one rounded fp32 add
+ *   g = v / 2 * (1 + erf(v / sqrt 2))  (if act == 1: the erf form of GELU, in fp64)
+ *   int8 output: q = clamp(round-half-even(g * out_scale), -128, 127)
+ *
+ * For act == 0 every step is one IEEE fp32 operation, so the result is exact
+ * and fixed: v32 holds v, q is decided in fp32 (one rounded multiply, then
+ * rintf).  For act == 1 the GELU is evaluated in fp64 from the fp32 v; pre
+ * holds g (fp64) and q is decided from g * out_scale in fp64.  Any of pre,
+ * v32, q may be NULL.
+ */
+static double gelu_erf(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }
+
+static int8_t sat_s8(double r) { return (int8_t)(r > 127.0 ? 127 : (r < -128.0 ? -128 : r)); }
+
+int oracle_epilogue_i8(const int32_t *acc, int64_t T, int64_t n_out, const float *scale,
+                       const float *bias, int act, float out_scale, double *pre, float *v32,
+                       int8_t *q) {
+    if (!acc || T < 0 || n_out <= 0 || (act != 0 && act != 1)) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t n = 0; n < n_out; ++n) {
+            const int64_t i = t * n_out + n;
+            volatile float v = (float)acc[i];
+            if (scale) v = v * scale[n];
+            if (bias) v = v + bias[n];
+            if (v32) v32[i] = v;
+            if (act == 1) {
+                const double g = gelu_erf((double)v);
+                if (pre) pre[i] = g;
+                if (q) q[i] = sat_s8(rint(g * (double)out_scale));
+            } else {
+                if (pre) pre[i] = (double)v;
+                if (q) {
+                    volatile float p = v * out_scale;
+                    q[i] = sat_s8((double)rintf(p));
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * The same output stage for the FP16/BF16 path, all in fp64 on the fp64
+ * accumulator (the kernel's fp32 result is compared against it within the
+ * tolerance):  g = act(acc * scale[n] + bias[n]).
+ */
+int oracle_epilogue_f(const double *acc, int64_t T, int64_t n_out, const float *scale,
+                      const float *bias, int act, double *pre) {
+    if (!acc || !pre || T < 0 || n_out <= 0 || (act != 0 && act != 1)) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t n = 0; n < n_out; ++n) {
+            const int64_t i = t * n_out + n;
+            double v = acc[i];
+            if (scale) v *= (double)scale[n];
+            if (bias) v += (double)bias[n];
+            pre[i] = act == 1 ? gelu_erf(v) : v;
+        }
+    }
+    return 0;
+}
+
+/* GELU alone, for the pins (closed forms of the normal CDF). */
+double oracle_gelu(double x) { return gelu_erf(x); }

@@ -271,3 +271,88 @@ def test_bf16_decoder_all_finite_patterns():
     Y = oracle.gemm(one, W, dtype="bf16")[0]
     want = torch.from_numpy(W[:, 0].view(np.int16).copy()).view(torch.bfloat16).double().numpy()
     assert np.array_equal(Y, want)
+
+
+# ------------------------------------------------------------------ fused output stage
+
+def _golden_epilogue():
+    with open(os.path.join(os.path.dirname(__file__), "golden", "epilogue_hand.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", _golden_epilogue()["cases"], ids=lambda c: c["name"])
+def test_epilogue_hand_cases(case):
+    acc = np.array(case["acc"], dtype=np.int32)
+    sc = None if case["scale"] is None else np.array(case["scale"], dtype=np.float32)
+    bi = None if case["bias"] is None else np.array(case["bias"], dtype=np.float32)
+    exp = np.array(case["expected"])
+    if "out_scale_per_case" in case:  # one column at a time, each with its own output scale
+        for j, os_ in enumerate(case["out_scale_per_case"]):
+            r = oracle.epilogue(acc[:, j:j + 1], sc, bi, case["act"], case["out"], os_)
+            assert int(r["q"][0, 0]) == int(exp[0, j])
+        return
+    r = oracle.epilogue(acc, sc, bi, case["act"], case["out"], case["out_scale"])
+    if case["out"] == "int8":
+        assert np.array_equal(r["q"], exp.astype(np.int8))
+        assert np.array_equal(r["exact"], exp.astype(np.int8))
+    else:
+        assert np.array_equal(r["exact"], exp.astype(np.float32))
+
+
+def test_gelu_matches_normal_cdf_table():
+    g = _golden_epilogue()["normal_cdf"]
+    for x, phi in zip(g["x"], g["phi"]):
+        assert abs(oracle.gelu(x) - x * phi) <= 1e-15 * x
+        assert abs(oracle.gelu(-x) - (-x * (1.0 - phi))) <= 1e-15 * x
+    assert oracle.gelu(0.0) == 0.0
+
+
+def test_gelu_odd_part_is_identity():
+    # erf is odd, so GELU(x) - GELU(-x) = x/2 (1 + erf) + x/2 (1 - erf) = x
+    for x in np.linspace(-8, 8, 161):
+        assert abs((oracle.gelu(x) - oracle.gelu(-x)) - x) <= 4e-16 * max(1.0, abs(x))
+    # far tails: GELU(x) -> x and GELU(-x) -> 0
+    assert oracle.gelu(12.0) == 12.0 and abs(oracle.gelu(-12.0)) < 1e-30
+
+
+def test_epilogue_int8_saturating_cast_closed_form():
+    rng = np.random.default_rng(3)
+    acc = rng.integers(-400, 400, size=(7, 33), dtype=np.int64).astype(np.int32)
+    r = oracle.epilogue(acc, out="int8")
+    assert np.array_equal(r["q"], np.clip(acc, -128, 127).astype(np.int8))
+    b = rng.integers(-50, 50, size=33).astype(np.float32)  # integer biases: exact sums
+    r = oracle.epilogue(acc, bias=b, out="int8")
+    assert np.array_equal(r["q"], np.clip(acc + b.astype(np.int64), -128, 127).astype(np.int8))
+
+
+def test_epilogue_per_channel_indexing():
+    # scale and bias are per output channel (column), never per token (row)
+    acc = np.arange(12, dtype=np.int32).reshape(3, 4)
+    sc = np.array([1, 2, 4, 8], dtype=np.float32)
+    bi = np.array([0, 100, 200, 300], dtype=np.float32)
+    r = oracle.epilogue(acc, sc, bi, out="float32")
+    want = np.array([[acc[t, n] * 2 ** n + 100 * n for n in range(4)] for t in range(3)], dtype=np.float32)
+    assert np.array_equal(r["exact"], want)
+    rf = oracle.epilogue(acc.astype(np.float64), sc, bi)
+    assert np.array_equal(rf["pre"], want.astype(np.float64))
+
+
+def test_epilogue_narrow_float_outputs_round_to_nearest_even():
+    # fp16 spacing is 2 in [2048, 4096): 2049 is halfway between 2048 and 2050 -> 2048 (even
+    # significand), 2051 between 2050 and 2052 -> 2052; 257 and 259 are exact.
+    # bf16 spacing is 16 at 2048 and 2 in [256, 512): 2049, 2051 -> 2048; 257 (halfway between
+    # 256 and 258) -> 256; 259 (halfway between 258 and 260) -> 260.
+    acc = np.array([[2049, 2051, 257, 259]], dtype=np.int32)
+    h = oracle.epilogue(acc, out="float16")["exact"]
+    assert h.tolist() == [[2048.0, 2052.0, 257.0, 259.0]]
+    b = oracle.epilogue(acc, out="bfloat16")["exact"]
+    vals = (b.astype(np.uint32) << 16).view(np.float32)
+    assert vals.tolist() == [[2048.0, 2048.0, 256.0, 260.0]]
+
+
+def test_epilogue_rejects_bad_arguments():
+    acc = np.zeros((2, 2), dtype=np.int32)
+    with pytest.raises(ValueError):
+        oracle.epilogue(acc, act="relu")
+    with pytest.raises(ValueError):
+        oracle.epilogue(acc.astype(np.float64), out="int8")
