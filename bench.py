@@ -212,7 +212,7 @@ def run_reference(args, rank: int) -> None:
 # --------------------------------------------------------------------------- other workloads
 
 
-def roofline_point(l, us: float, pk: dict) -> dict:
+def roofline_point(l, us: float, pk: dict, out_es: int | None = None, biased: bool = False) -> dict:
     """Roofline of one problem: t = max(ops / tensor peak, bytes / HBM peak).
 
     Tensor peaks derive from the measured bf16 dense peak with NVIDIA's nominal
@@ -223,7 +223,7 @@ def roofline_point(l, us: float, pk: dict) -> dict:
     tc_peak = dense_peak * (2.0 if sparse else 1.0)
     ops = l.dense_ops()
     t_tc = ops / (tc_peak * 1e12) * 1e6
-    bytes_ = alg_bytes_any(l)
+    bytes_ = alg_bytes_any(l, out_es, biased)
     t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9) * 1e6
     t_roof = max(t_tc, t_hbm)
     return {"us": round(us, 2), "dense_eq_tops": round(ops / us / 1e6, 1),
@@ -231,14 +231,17 @@ def roofline_point(l, us: float, pk: dict) -> dict:
             "frac": round(t_roof / us, 3)}
 
 
-def alg_bytes_any(l) -> int:
-    """Algorithmic bytes of one SpMM launch for any dtype/output."""
+def alg_bytes_any(l, out_es: int | None = None, biased: bool = False) -> int:
+    """Algorithmic bytes of one SpMM launch for any dtype/output (out_es: bytes
+    per output element when not the default of the dtype)."""
     import math
     es = 1 if l.dtype == inputs.INT8 else 2
     kept = l.n_out * (l.K // l.M) * l.N
     wbytes = (kept * es + (kept * math.ceil(math.log2(l.M)) + 7) // 8) if l.N != l.M else l.n_out * l.K * es
-    out_es = (4 if l.dtype == inputs.INT8 else 2)
-    return l.T * l.K * es + wbytes + l.T * l.n_out * out_es + (4 * l.n_out if l.scaled else 0)
+    if out_es is None:
+        out_es = 4 if l.dtype == inputs.INT8 else 2
+    return (l.T * l.K * es + wbytes + l.T * l.n_out * out_es + (4 * l.n_out if l.scaled else 0)
+            + (4 * l.n_out if biased else 0))
 
 
 def run_config(name: str, args) -> None:
@@ -252,6 +255,9 @@ def run_config(name: str, args) -> None:
         ls, desc = inputs.vit_l_fp16(), "ViT-L/16 linears, batch 32 (T=6304), FP16, N:M in {1:4,2:4,2:8}"
     elif name == "swin":
         ls, desc = inputs.swin_t_int8(), "Swin-T linears per stage, batch 128, INT8 + scale, N:M in {2:4,2:8}"
+    elif name == "int8out":
+        ls, desc = inputs.vit_b_int8(), ("ViT-B/16 INT8 linear set, batch 64 (T=12608), N:M in {1:4,2:4,2:8,4:8}, "
+                                         "fused int8 output: per-channel scale + bias, GELU after fc1, requantised")
     elif name in ("mixed1", "mixed256"):
         T = 197 if name == "mixed1" else 50432
         ls, desc = inputs.vit_b_mixed(T), f"all 48 ViT-B linears at T={T}, per-layer N:M from {{dense,4:8,2:4,2:8,1:4}}"
@@ -259,19 +265,28 @@ def run_config(name: str, args) -> None:
         raise SystemExit(f"unknown config {name}")
     stream = torch.cuda.current_stream()
     probs = []
+    int8out = name == "int8out"
     for l in ls:
         W, X, sc = l.weight().cuda(), l.activation().cuda(), l.scale()
         sc = None if sc is None else sc.cuda()
         h = nm.nm_compress(W, l.N, l.M)
-        Y = torch.empty((l.T, l.n_out), dtype=nm.out_dtype(h, sc is not None), device="cuda")
-        probs.append((l, W, X, sc, h, Y))
+        if int8out:  # per-channel bias; GELU after fc1; one int8 step = 10 output units
+            bias = inputs.normal_f32((l.n_out,), 5.0, l.seed + 3).cuda()
+            act = "gelu" if l.name.endswith("fc1") else "none"
+            Y = torch.empty((l.T, l.n_out), dtype=torch.int8, device="cuda")
+            call = (lambda st, h=h, X=X, Y=Y, sc=sc, bias=bias, act=act:
+                    nm.nm_spmm_ex(h, X, Y=Y, scale=sc, bias=bias, act=act, out="int8", out_scale=0.1, stream=st))
+        else:
+            Y = torch.empty((l.T, l.n_out), dtype=nm.out_dtype(h, sc is not None), device="cuda")
+            call = (lambda st, h=h, X=X, Y=Y, sc=sc: nm.nm_spmm(h, X, Y=Y, scale=sc, stream=st))
+        probs.append((l, W, X, sc, h, Y, call))
     torch.cuda.synchronize()
 
     def run_all(evs=None):
-        for i, (l, W, X, sc, h, Y) in enumerate(probs):
+        for i, p in enumerate(probs):
             if evs is not None:
                 evs[i][0].record(stream)
-            nm.nm_spmm(h, X, Y=Y, scale=sc, stream=stream)
+            p[6](stream)
             if evs is not None:
                 evs[i][1].record(stream)
 
@@ -295,17 +310,17 @@ def run_config(name: str, args) -> None:
 
     def seq_body(cap):
         for r in range(reps):
-            for (l, W, X, sc, h, Y) in probs:
-                nm.nm_spmm(h, X, Y=Y, scale=sc, stream=cap)
+            for p in probs:
+                p[6](cap)
 
     evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in probs]
            for _ in range(reps)]
 
     def per_body(cap):
         for r in range(reps):
-            for i, (l, W, X, sc, h, Y) in enumerate(probs):
+            for i, p in enumerate(probs):
                 evs[r][i][0].record(cap)
-                nm.nm_spmm(h, X, Y=Y, scale=sc, stream=cap)
+                p[6](cap)
                 evs[r][i][1].record(cap)
 
     g = capture(seq_body)
@@ -322,9 +337,9 @@ def run_config(name: str, args) -> None:
         if nm.nm_device_status(h) != nm.NM_OK:
             raise RuntimeError(nm.nm_last_error())
     per = []
-    for i, (l, W, X, sc, h, Y) in enumerate(probs):
+    for i, (l, W, X, sc, h, Y, _) in enumerate(probs):
         us = statistics.median(evs[r][i][0].elapsed_time(evs[r][i][1]) * 1e3 for r in range(reps))
-        rp = roofline_point(l, us, pk)
+        rp = roofline_point(l, us, pk, 1 if int8out else None, int8out)
         # same-shape cuBLAS dense GEMM through torch (context)
         if l.dtype == inputs.INT8 and l.T > 16:
             fn = (lambda X=X, W=W: torch._int_mm(X, W.t()))
@@ -371,7 +386,7 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
-    ap.add_argument("--config", default=None, choices=["single", "vitl", "swin", "mixed1", "mixed256"],
+    ap.add_argument("--config", default=None, choices=["single", "vitl", "swin", "mixed1", "mixed256", "int8out"],
                     help="measure another workload (one JSON line) instead of the default ViT-B INT8 set")
     ap.add_argument("--only", action="append", default=[],
                     help="restrict to problems like vitb.fc1/2:4 (profiling a single kernel shape)")

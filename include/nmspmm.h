@@ -136,6 +136,59 @@ nm_status nm_spmm(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
                   const float* scale_dev, void* stream);
 
 /*
+ * Fused output stage of nm_spmm_ex.  The paper stops at the MMA (section 4.2)
+ * and does not discuss the output stage; this is the library's definition.
+ * Per output element, in fp32, each step rounded to nearest:
+ *   v = acc                         INT8: (float)acc; FP16/BF16: the fp32 sum
+ *   v = v * scale[n]                if scale != NULL
+ *   v = v + bias[n]                 if bias != NULL
+ *   v = v/2 * (1 + erf(v/sqrt 2))   if act == NM_ACT_GELU (erf form of GELU)
+ * then stored as the output type:
+ *   NM_OUT_FP32                     v
+ *   NM_OUT_FP16 / NM_OUT_BF16       v rounded to nearest even
+ *   NM_OUT_INT8                     clamp(round_half_even(v * out_scale), -128, 127)
+ *   NM_OUT_INT32                    the raw INT8 accumulator (no scale, bias
+ *                                   or activation allowed)
+ *   NM_OUT_DEFAULT                  INT8: INT32 when scale, bias and act are
+ *                                   all absent, else FP32; FP16/BF16: the
+ *                                   input's type.
+ * With act == NM_ACT_NONE and an INT8 handle the result is exactly fixed; the
+ * GELU uses the device's erff, so it is within erff's error bound.
+ */
+typedef enum {
+  NM_OUT_DEFAULT = 0,
+  NM_OUT_INT32 = 1,
+  NM_OUT_FP32 = 2,
+  NM_OUT_FP16 = 3,
+  NM_OUT_BF16 = 4,
+  NM_OUT_INT8 = 5
+} nm_out_type;
+
+typedef enum { NM_ACT_NONE = 0, NM_ACT_GELU = 1 } nm_act;
+
+typedef struct nm_epilogue {
+  nm_out_type out;     /* element type of Y */
+  nm_act act;          /* activation after scale and bias */
+  const float* scale;  /* device float32 [n_out], 4-byte aligned, or NULL */
+  const float* bias;   /* device float32 [n_out], 4-byte aligned, or NULL */
+  float out_scale;     /* NM_OUT_INT8 only: multiplier before rounding; finite and > 0 */
+} nm_epilogue;
+
+/*
+ * nm_spmm_ex -- nm_spmm with the fused output stage above: Y = out(act(
+ * (X . Wm^T) * scale + bias)).  Arguments, alignment, the no-op for T == 0,
+ * the workspace rule and the never-synchronise rule are those of nm_spmm; Y_dev
+ * holds elements of the chosen output type.  ep == NULL is nm_spmm with no
+ * scale.
+ * Errors: NM_ERR_INVALID for an unknown out/act value, NM_OUT_INT32 together
+ * with scale, bias or act, a misaligned scale/bias, or NM_OUT_INT8 with an
+ * out_scale that is not finite and positive; NM_ERR_UNSUPPORTED for
+ * NM_OUT_INT32 or NM_OUT_INT8 on an FP16/BF16 handle.
+ */
+nm_status nm_spmm_ex(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
+                     const nm_epilogue* ep, void* stream);
+
+/*
  * nm_decompress -- write the masked dense weight Wm [n_out][k] (dtype of the
  * handle) decoded from the packed operand image the SpMM kernel reads, so the
  * image can be checked against the top-N rule.  W_dev_out 16-byte aligned.

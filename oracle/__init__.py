@@ -222,7 +222,8 @@ def epilogue(acc: np.ndarray, scale: np.ndarray | None = None, bias: np.ndarray 
             if out == "float32":
                 res["exact"] = v32
             elif out == "float16":
-                res["exact"] = v32.astype(np.float16)
+                with np.errstate(over="ignore"):  # beyond the fp16 range rounds to +-inf, as defined
+                    res["exact"] = v32.astype(np.float16)
             else:
                 import torch
                 res["exact"] = torch.from_numpy(v32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)

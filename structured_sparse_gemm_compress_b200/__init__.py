@@ -24,7 +24,7 @@ _TORCH_DT = {torch.int8: NM_INT8, torch.float16: NM_FP16, torch.bfloat16: NM_BF1
 _ELEM = {NM_INT8: torch.int8, NM_FP16: torch.float16, NM_BF16: torch.bfloat16}
 
 # Every symbol include/nmspmm.h declares.
-EXPORTS = ("nm_compress", "nm_recompress", "nm_spmm", "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
+EXPORTS = ("nm_compress", "nm_recompress", "nm_spmm", "nm_spmm_ex", "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
            "nm_device_status", "nm_destroy", "nm_last_error", "nm_version", "nm_test_spmm_skip_stage")
 
 
@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         L.nm_recompress.argtypes = [vp, vp, vp]
         L.nm_spmm.argtypes = [vp, vp, i64, vp, vp, vp]
         L.nm_spmm_noalloc.argtypes = [vp, vp, i64, vp, vp, vp]
+        L.nm_spmm_ex.argtypes = [vp, vp, i64, vp, ctypes.POINTER(NMEpilogue), vp]
         L.nm_test_spmm_skip_stage.argtypes = [vp, vp, i64, vp, vp, vp, i32, i64]
         L.nm_decompress.argtypes = [vp, vp, vp]
         L.nm_export.argtypes = [vp, vp, vp]
@@ -155,6 +156,52 @@ def nm_spmm(h: NMHandle, X: torch.Tensor, Y: torch.Tensor | None = None, scale: 
     if scale is not None and (scale.dtype != torch.float32 or scale.numel() != h.n_out or not scale.is_cuda):
         raise ValueError("scale must be a CUDA float32 tensor of n_out elements")
     _check(lib().nm_spmm(h.raw, _ptr(X), T, _ptr(Y), _ptr(scale), _stream(stream)))
+    return Y
+
+
+class NMEpilogue(ctypes.Structure):
+    """``nm_epilogue`` of include/nmspmm.h."""
+    _fields_ = [("out", ctypes.c_int), ("act", ctypes.c_int), ("scale", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("out_scale", ctypes.c_float)]
+
+
+OUT_TYPES = {"default": 0, "int32": 1, "float32": 2, "float16": 3, "bfloat16": 4, "int8": 5}
+ACTS = {"none": 0, "gelu": 1}
+_OUT_TORCH = {"int32": torch.int32, "float32": torch.float32, "float16": torch.float16,
+              "bfloat16": torch.bfloat16, "int8": torch.int8}
+
+
+def resolve_out(h: NMHandle, out: str, scale, bias, act: str) -> str:
+    """The output type ``NM_OUT_DEFAULT`` stands for, by the header's rule."""
+    if out != "default":
+        return out
+    if h.dtype == torch.int8:
+        return "int32" if scale is None and bias is None and act == "none" else "float32"
+    return "float16" if h.dtype == torch.float16 else "bfloat16"
+
+
+def nm_spmm_ex(h: NMHandle, X: torch.Tensor, Y: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+               bias: torch.Tensor | None = None, act: str = "none", out: str = "default",
+               out_scale: float = 1.0, stream=None) -> torch.Tensor:
+    """Y = out(act(X @ Wm^T * scale + bias)) with the fused output stage of
+    ``nm_spmm_ex`` (include/nmspmm.h).  ``out`` is one of ``OUT_TYPES``, ``act``
+    one of ``ACTS``.  Only argument marshalling happens here."""
+    if X.dtype != h.dtype or not X.is_cuda or not X.is_contiguous() or X.dim() != 2 or X.shape[1] != h.k:
+        raise ValueError("X must be a contiguous CUDA [T, k] tensor of the handle's dtype")
+    if out not in OUT_TYPES or act not in ACTS:
+        raise ValueError(f"out must be one of {tuple(OUT_TYPES)}, act one of {tuple(ACTS)}")
+    for name, v in (("scale", scale), ("bias", bias)):
+        if v is not None and (v.dtype != torch.float32 or v.numel() != h.n_out or not v.is_cuda):
+            raise ValueError(f"{name} must be a CUDA float32 tensor of n_out elements")
+    T = X.shape[0]
+    res = resolve_out(h, out, scale, bias, act)
+    want = _OUT_TORCH[res]
+    if Y is None:
+        Y = torch.empty((T, h.n_out), dtype=want, device=X.device)
+    elif Y.dtype != want or tuple(Y.shape) != (T, h.n_out) or not Y.is_contiguous():
+        raise ValueError(f"Y must be a contiguous [{T}, {h.n_out}] {want} tensor")
+    ep = NMEpilogue(OUT_TYPES[out], ACTS[act], _ptr(scale), _ptr(bias), float(out_scale))
+    _check(lib().nm_spmm_ex(h.raw, _ptr(X), T, _ptr(Y), ctypes.byref(ep), _stream(stream)))
     return Y
 
 

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -264,8 +265,22 @@ nm_status check_handle(const nm_handle* h) {
   return NM_OK;
 }
 
+// Output stage chosen at run time (nm_spmm_ex); out_ty < 0: the fixed stage of nm_spmm.
+struct EpiReq {
+  int out_ty = -1;  // nm::OUT_F32 / F16 / BF16 / I8
+  const float* bias = nullptr;
+  int act = nm::ACT_NONE;
+  float out_scale = 1.0f;
+};
+
+int out_elem_bytes(const nm_handle* h, const EpiReq* ep) {
+  if (ep && ep->out_ty >= 0)
+    return ep->out_ty == nm::OUT_I8 ? 1 : (ep->out_ty == nm::OUT_F32 ? 4 : 2);
+  return h->dt == nm::DT_I8 ? 4 : 2;
+}
+
 nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, const float* scale, void* stream,
-                    int inject_skip, unsigned long long timeout_ns) {
+                    int inject_skip, unsigned long long timeout_ns, const EpiReq* ep = nullptr) {
   g_err.clear();
   nm_status st = check_handle(hc);
   if (st != NM_OK) return st;
@@ -279,7 +294,7 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   if ((h->k * es) % 16 != 0)
     return fail(NM_ERR_UNSUPPORTED, "k * sizeof(dtype) must be a multiple of 16 bytes (k=%lld)", (long long)h->k);
   if (scale && !aligned(scale, 4)) return fail(NM_ERR_INVALID, "scale must be 4-byte aligned");
-  const size_t ybytes = (size_t)T * h->n_out * ((h->dt == nm::DT_I8) ? 4 : 2);
+  const size_t ybytes = (size_t)T * h->n_out * out_elem_bytes(h, ep);
   const size_t xbytes = (size_t)T * h->k * es;
   const uintptr_t xs = (uintptr_t)X, ys = (uintptr_t)Y;
   if (xs < ys + ybytes && ys < xs + xbytes) return fail(NM_ERR_INVALID, "Y overlaps X");
@@ -305,6 +320,10 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   a.timeout_ns = timeout_ns;
   a.inject_skip = inject_skip;
   a.w_tma = (h->has_tmw && env_int("NMSPMM_W_BULK", 0) == 0) ? 1 : 0;
+  a.out_ty = ep ? ep->out_ty : -1;
+  a.bias = ep ? ep->bias : nullptr;
+  a.act = ep ? ep->act : nm::ACT_NONE;
+  a.out_scale = ep ? ep->out_scale : 1.0f;
 #ifdef NM_TRACE
   // timeline builds only: device buffer of grid * kTraceStride int64 given as an integer address
   if (const char* tp = getenv("NMSPMM_TRACE_PTR")) a.trace = reinterpret_cast<long long*>(strtoull(tp, nullptr, 0));
@@ -336,11 +355,12 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   }
   int oes, oty;
   out_type(h, scale != nullptr, &oes, &oty);
-  const int ych = p.pair ? ((p.bn / 2) % 32 == 0 ? 32 : 16) : std::min(32, p.bn / 2);  // epilogue chunk
+  const int wcols = p.bn / nm::epw_for(false);  // token columns per epilogue warp; the TMA-store box
+  const int ych = p.pair ? (wcols % 32 == 0 ? 32 : wcols % 16 == 0 ? 16 : 8) : std::min(32, wcols);
   // Direct stores measured faster than staged TMA stores (they keep the TMA unit
   // for operand loads); the TMA-store epilogue remains selectable.
   a.tma_store = 0;
-  if (env_int("NMSPMM_TMA_STORE", 0)) a.tma_store = make_y_map(h, Y, T, oes, oty, ych, &st) ? 1 : 0;
+  if (env_int("NMSPMM_TMA_STORE", 0) && a.out_ty < 0) a.tma_store = make_y_map(h, Y, T, oes, oty, ych, &st) ? 1 : 0;
   if (st != NM_OK) return st;
   cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "launch SpMM kernel");
@@ -454,6 +474,41 @@ nm_status nm_recompress(nm_handle* h, const void* W_dev, void* stream) {
 nm_status nm_spmm(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev, const float* scale_dev,
                   void* stream) {
   return spmm_impl(h, X_dev, T, Y_dev, scale_dev, stream, -1, 1000000000ull);
+}
+
+nm_status nm_spmm_ex(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev, const nm_epilogue* ep,
+                     void* stream) {
+  g_err.clear();
+  if (!ep) return spmm_impl(h, X_dev, T, Y_dev, nullptr, stream, -1, 1000000000ull);
+  nm_status st = check_handle(h);
+  if (st != NM_OK) return st;
+  if ((int)ep->out < 0 || (int)ep->out > 5) return fail(NM_ERR_INVALID, "unknown output type %d", (int)ep->out);
+  if ((int)ep->act < 0 || (int)ep->act > 1) return fail(NM_ERR_INVALID, "unknown activation %d", (int)ep->act);
+  if ((ep->scale && !aligned(ep->scale, 4)) || (ep->bias && !aligned(ep->bias, 4)))
+    return fail(NM_ERR_INVALID, "scale and bias must be 4-byte aligned");
+  const bool plain = !ep->scale && !ep->bias && ep->act == NM_ACT_NONE;
+  const bool int_in = h->dt == nm::DT_I8;
+  nm_out_type out = ep->out;
+  if (out == NM_OUT_DEFAULT)
+    out = int_in ? (plain ? NM_OUT_INT32 : NM_OUT_FP32) : (h->dt == nm::DT_F16 ? NM_OUT_FP16 : NM_OUT_BF16);
+  if (!int_in && (out == NM_OUT_INT32 || out == NM_OUT_INT8))
+    return fail(NM_ERR_UNSUPPORTED, "integer outputs need an INT8 handle");
+  if (out == NM_OUT_INT32 && !plain)
+    return fail(NM_ERR_INVALID, "NM_OUT_INT32 is the raw accumulator: no scale, bias or activation");
+  if (out == NM_OUT_INT8 && !(std::isfinite(ep->out_scale) && ep->out_scale > 0.0f))
+    return fail(NM_ERR_INVALID, "out_scale must be finite and positive for NM_OUT_INT8");
+  // The fixed stages of nm_spmm compute the same values; use them where they apply.
+  const bool fixed = ep->act == NM_ACT_NONE && !ep->bias &&
+                     ((int_in && out == NM_OUT_INT32) || (int_in && out == NM_OUT_FP32 && ep->scale) ||
+                      (h->dt == nm::DT_F16 && out == NM_OUT_FP16) || (h->dt == nm::DT_BF16 && out == NM_OUT_BF16));
+  if (fixed) return spmm_impl(h, X_dev, T, Y_dev, ep->scale, stream, -1, 1000000000ull);
+  EpiReq r;
+  r.out_ty = out == NM_OUT_FP32 ? nm::OUT_F32 : out == NM_OUT_FP16 ? nm::OUT_F16 : out == NM_OUT_BF16 ? nm::OUT_BF16
+                                                                                                      : nm::OUT_I8;
+  r.bias = ep->bias;
+  r.act = ep->act == NM_ACT_GELU ? nm::ACT_GELU : nm::ACT_NONE;
+  r.out_scale = ep->out_scale;
+  return spmm_impl(h, X_dev, T, Y_dev, ep->scale, stream, -1, 1000000000ull, &r);
 }
 
 nm_status nm_test_spmm_skip_stage(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
@@ -579,7 +634,8 @@ nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y
   }
   int oes, oty;
   out_type(h, scale != nullptr, &oes, &oty);
-  const int ych = p.pair ? ((p.bn / 2) % 32 == 0 ? 32 : 16) : std::min(32, p.bn / 2);  // epilogue chunk
+  const int wcols = p.bn / nm::epw_for(false);  // token columns per epilogue warp; the TMA-store box
+  const int ych = p.pair ? (wcols % 32 == 0 ? 32 : wcols % 16 == 0 ? 16 : 8) : std::min(32, wcols);
   // Direct stores measured faster than staged TMA stores (they keep the TMA unit
   // for operand loads); the TMA-store epilogue remains selectable.
   a.tma_store = 0;

@@ -36,7 +36,8 @@ namespace nm {
 
 enum : int { DT_I8 = 0, DT_F16 = 1, DT_BF16 = 2 };
 enum : int { IMG_SP24 = 0, IMG_DENSE = 1 };
-enum : int { OUT_I32 = 0, OUT_F32 = 1, OUT_F16 = 2, OUT_BF16 = 3 };  // output element of a launch
+enum : int { OUT_I32 = 0, OUT_F32 = 1, OUT_F16 = 2, OUT_BF16 = 3, OUT_I8 = 4 };  // output element of a launch
+enum : int { ACT_NONE = 0, ACT_GELU = 1 };  // activation of the fused output stage
 
 constexpr int kRows = 128;          // channel rows per tile (MMA M)
 constexpr int kAtomBytes = 16384;   // 128 rows x 128 B swizzled atom
@@ -394,6 +395,14 @@ __device__ __forceinline__ void bulk_wait() {
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA).
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
 }
 
 // 32 lanes x 16 consecutive 32-bit columns.

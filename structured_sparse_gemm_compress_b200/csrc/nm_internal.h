@@ -60,6 +60,13 @@ struct Plan {
   int pair = 0;       // 1: CTA-pair kernel (M = 256 per MMA); grid counts pairs
 };
 
+// Epilogue warps per TMEM lane quarter (each owns BN / epw token columns of a
+// tile): 2 for the fixed output stages, 4 for the runtime output stage, whose
+// longer per-element work needs more warps to hide its latencies.  The fixed
+// stages keep the smaller CTA so that other kernels (weight re-packs) can share
+// the SM.
+constexpr int epw_for(bool runtime_stage) { return runtime_stage ? 4 : 2; }
+
 // Largest number of INT8 k-blocks (256 dense k each) the X-stationary mode keeps resident.
 constexpr int kXsMaxKb = 3;
 
@@ -75,6 +82,13 @@ struct SpmmArgs {
   int tma_store;      // 1: epilogue writes Y with TMA tensor stores (tmY valid)
   int w_tma;          // 1: packed chunks arrive by 2-D tensor copy (tmW valid), else one bulk copy
   int inject_skip;    // test hook: producer omits the stage with this index (-1: never)
+  // Fused output stage chosen at run time (kernels built with the runtime output
+  // stage only): element type OUT_F32/F16/BF16/I8, per-channel bias (or null),
+  // activation ACT_*, and the multiplier applied before int8 rounding.
+  int out_ty = -1;
+  const float* bias = nullptr;
+  int act = 0;
+  float out_scale = 1.0f;
   long long* trace;   // timeline buffer, only written by builds compiled with NM_TRACE
 };
 

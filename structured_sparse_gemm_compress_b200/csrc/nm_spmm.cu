@@ -18,16 +18,15 @@
 // = token; the epilogue therefore stores 32 consecutive channels of one token
 // per warp instruction (128 B, coalesced) without a transpose.
 //
-// CTA = 10 warps, one persistent CTA per SM:
+// CTA = 2 + 4 * epw warps, one persistent CTA per SM:
 //   warp 0      producer: one bulk copy of the packed weight chunk (values +
 //               positions) and two 2-D tensor copies of X per stage;
 //   warp 1      TMEM owner and MMA issuer (one thread): copies the positions
 //               into TMEM (tcgen05.cp) and issues tcgen05.mma(.sp);
-//   warps 2..9  epilogue, two warps per TMEM lane quarter (one per half of the
-//               token columns): tcgen05.ld, optional per-channel scale, then
-//               either a staged tile in shared memory written by a TMA tensor
-//               store (3 instructions per element) or, when Y's row pitch is
-//               not a multiple of 16 bytes, direct coalesced stores.
+//   warps 2..   epilogue, epw warps per TMEM lane quarter (each owning BN/epw
+//               token columns): tcgen05.ld, the output stage, then coalesced
+//               direct stores (one 32-channel run of a token per instruction)
+//               or, optionally, a staged tile written by a TMA tensor store.
 // Two TMEM accumulators let the epilogue of one tile overlap the mainloop of
 // the next.  Every wait is bounded; on a timeout the kernel records an error
 // word, drains its own copies and MMAs, frees TMEM and returns.
@@ -37,17 +36,23 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 namespace nm {
 
 
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemBudget = 227 * 1024 - 1024;  // dynamic shared memory after 1 KB alignment slack
 
 // OUT template parameter: bits 0-1 = output element (OUT_*), bit 2 = direct-store
-// epilogue (no shared-memory staging, which leaves room for more pipeline stages).
+// epilogue (no shared-memory staging, which leaves room for more pipeline stages),
+// bit 3 = runtime output stage (scale, bias, activation and element type read from
+// SpmmArgs; always with direct stores).
 constexpr int kOutDirect = 4;
+constexpr int kOutEpi = 8;
 constexpr int out_bytes(int out) { return ((out & 3) == OUT_I32 || (out & 3) == OUT_F32) ? 4 : 2; }
+// Epilogue warps and CTA size of a kernel with output code OUT.
+constexpr int epi_warps(int out) { return 4 * epw_for((out & kOutEpi) != 0); }
+constexpr int cta_threads(int out) { return 64 + 32 * epi_warps(out); }
 
 // Kernel configuration.  XKB = 0: streaming mode, every stage carries a packed
 // weight chunk and the matching X boxes.  XKB > 0: X-stationary mode, the
@@ -71,25 +76,27 @@ struct Cfg {
   static constexpr int COLS_NEEDED = 2 * BN + 2 * E_COLS;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 : COLS_NEEDED <= 128 ? 128
                                    : COLS_NEEDED <= 256 ? 256 : 512;
-  // epilogue: each warp owns BN/2 token columns of its lane quarter, in chunks of CH
-  static constexpr int HALF = BN / 2;
-  static constexpr int CH = HALF >= 32 ? 32 : HALF;
-  static constexpr int NCH = HALF / CH;
+  // epilogue: each warp owns BN/epw token columns of its lane quarter, in chunks of CH
+  static constexpr int EPI_WARPS = epi_warps(OUT);
+  static constexpr int THREADS = cta_threads(OUT);
+  static constexpr int WCOLS = BN / (EPI_WARPS / 4);
+  static constexpr int CH = WCOLS >= 32 ? 32 : WCOLS;
+  static constexpr int NCH = WCOLS / CH;
   static constexpr int OES = out_bytes(OUT);
   static constexpr int EPI_BUF = CH * 32 * OES;     // one staged [CH tokens][32 channels] tile
   static constexpr int AVAIL = kSmemBudget - X_BYTES;
   // two staging buffers per warp unless that would leave fewer stages than wanted
   static constexpr int WANT = XS ? 4 : 3;
   static constexpr bool TS = (OUT & kOutDirect) == 0;   // TMA-store epilogue with staging
-  static constexpr int EPI_NB = (AVAIL - 2 * kEpiWarps * EPI_BUF) / STAGE >= WANT ? 2 : 1;
-  static constexpr int EPI_BYTES = TS ? EPI_NB * kEpiWarps * EPI_BUF : 0;
+  static constexpr int EPI_NB = (AVAIL - 2 * EPI_WARPS * EPI_BUF) / STAGE >= WANT ? 2 : 1;
+  static constexpr int EPI_BYTES = TS ? EPI_NB * EPI_WARPS * EPI_BUF : 0;
   static constexpr int STAGES_FIT = (AVAIL - EPI_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int SMEM = STAGES * STAGE + X_BYTES + EPI_BYTES + 1024;
   static_assert(STAGE % 1024 == 0 && B_KBLK % 1024 == 0, "stages keep 1024-byte alignment");
   static_assert(STAGES >= 2, "need at least two stages");
   static_assert(COLS_NEEDED <= 512, "tensor memory overflow");
-  static_assert(HALF % CH == 0 && CH % 16 == 0, "epilogue chunking");
+  static_assert(WCOLS % CH == 0 && CH % 8 == 0, "epilogue chunking");
 };
 
 // Instruction descriptor: A K-major (sparse or dense), B K-major, M = 128.
@@ -139,6 +146,13 @@ __device__ __forceinline__ Unit decode_unit(int u, const SpmmArgs& a) {
   w.kb0 = w.z * a.kb_per_split;
   w.kb1 = min(a.n_kb, w.kb0 + a.kb_per_split);
   return w;
+}
+
+// clamp(round-half-even(x), -128, 127) in one conversion instruction (NaN -> 0).
+__device__ __forceinline__ int32_t rne_sat_s8(float x) {
+  int32_t q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(x));
+  return q;
 }
 
 // Output element from the 32-bit accumulator: int32; (float)acc * scale; or
@@ -196,6 +210,109 @@ __device__ __forceinline__ void store_out(void* Y, size_t i, uint32_t acc, float
   }
 }
 
+// ---- runtime output stage (OUT has kOutEpi)
+//
+// y = act(acc * scale[n] + bias[n]) in fp32, one rounding per step (scale and
+// bias only when given), then stored as fp32, fp16 or bf16 (round to nearest
+// even) or int8 (round half to even of y * out_scale, saturated to [-128, 127]).
+// The GELU is the erf form x/2 (1 + erf(x / sqrt 2)).
+struct EpiCh {  // per output channel
+  float s, b;
+};
+
+__device__ __forceinline__ float gelu_erf(float x) {
+  const float t = erff(__fmul_rn(x, 0.70710677f));  // fp32(1/sqrt(2))
+  return __fmul_rn(0.5f, __fmul_rn(x, __fadd_rn(1.0f, t)));
+}
+
+template <int DT>
+__device__ __forceinline__ float epi_value(uint32_t acc, const EpiCh& e, const SpmmArgs& a) {
+  float f = DT == DT_I8 ? __int2float_rn((int32_t)acc) : __uint_as_float(acc);
+  if (a.scale) f = __fmul_rn(f, e.s);
+  if (a.bias) f = __fadd_rn(f, e.b);
+  if (a.act == ACT_GELU) f = gelu_erf(f);
+  return f;
+}
+
+template <int OT>
+__device__ __forceinline__ void epi_put(void* Y, size_t i, float f, float out_scale) {
+  if constexpr (OT == OUT_F32) {
+    reinterpret_cast<float*>(Y)[i] = f;
+  } else if constexpr (OT == OUT_F16) {
+    reinterpret_cast<__half*>(Y)[i] = __float2half_rn(f);
+  } else if constexpr (OT == OUT_BF16) {
+    reinterpret_cast<__nv_bfloat16*>(Y)[i] = __float2bfloat16_rn(f);
+  } else {
+    reinterpret_cast<int8_t*>(Y)[i] = (int8_t)rne_sat_s8(__fmul_rn(f, out_scale));
+  }
+}
+
+// One channel's run of CH consecutive tokens (row stride n_out), the first
+// nvalid of them inside the output.  Two phases, so each optional step is one
+// uniform branch around one short loop (the GELU's code exists once): values
+// first, then one store loop per element type.
+template <int OT, int CH>
+__device__ __forceinline__ void epi_store_t(const SpmmArgs& a, const float (&f)[CH], size_t base, int nvalid) {
+  if constexpr (OT == OUT_F16 || OT == OUT_BF16) {
+    // one paired conversion (round to nearest even each) per two tokens
+    using T2 = typename std::conditional<OT == OUT_F16, __half2, __nv_bfloat162>::type;
+    using T1 = typename std::conditional<OT == OUT_F16, __half, __nv_bfloat16>::type;
+    T1* y = reinterpret_cast<T1*>(a.Y) + base;
+#pragma unroll
+    for (int j = 0; j < CH; j += 2) {
+      T2 p;
+      if constexpr (OT == OUT_F16)
+        p = __floats2half2_rn(f[j], f[j + 1]);
+      else
+        p = __floats2bfloat162_rn(f[j], f[j + 1]);
+      if (j < nvalid) y[(size_t)j * a.n_out] = p.x;
+      if (j + 1 < nvalid) y[(size_t)(j + 1) * a.n_out] = p.y;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < CH; ++j)
+      if (j < nvalid) epi_put<OT>(a.Y, base + (size_t)j * a.n_out, f[j], a.out_scale);
+  }
+}
+
+template <int DT, int CH>
+__device__ __forceinline__ void epi_run(const SpmmArgs& a, const EpiCh& e, const uint32_t (&r)[CH], size_t base,
+                                        int nvalid) {
+  float f[CH];
+#pragma unroll
+  for (int j = 0; j < CH; ++j) f[j] = DT == DT_I8 ? __int2float_rn((int32_t)r[j]) : __uint_as_float(r[j]);
+  if (a.scale) {
+#pragma unroll
+    for (int j = 0; j < CH; ++j) f[j] = __fmul_rn(f[j], e.s);
+  }
+  if (a.bias) {
+#pragma unroll
+    for (int j = 0; j < CH; ++j) f[j] = __fadd_rn(f[j], e.b);
+  }
+  if (a.act == ACT_GELU) {
+#pragma unroll
+    for (int j = 0; j < CH; ++j) f[j] = gelu_erf(f[j]);
+  }
+  switch (a.out_ty) {
+    case OUT_F16: epi_store_t<OUT_F16, CH>(a, f, base, nvalid); break;
+    case OUT_BF16: epi_store_t<OUT_BF16, CH>(a, f, base, nvalid); break;
+    case OUT_I8: epi_store_t<OUT_I8, CH>(a, f, base, nvalid); break;
+    default: epi_store_t<OUT_F32, CH>(a, f, base, nvalid); break;
+  }
+}
+
+// A single element (split-K reduction).
+template <int DT>
+__device__ __forceinline__ void epi_one(const SpmmArgs& a, const EpiCh& e, size_t i, uint32_t acc) {
+  const float f = epi_value<DT>(acc, e, a);
+  switch (a.out_ty) {
+    case OUT_F16: epi_put<OUT_F16>(a.Y, i, f, a.out_scale); break;
+    case OUT_BF16: epi_put<OUT_BF16>(a.Y, i, f, a.out_scale); break;
+    case OUT_I8: epi_put<OUT_I8>(a.Y, i, f, a.out_scale); break;
+    default: epi_put<OUT_F32>(a.Y, i, f, a.out_scale); break;
+  }
+}
+
 // Sum of split partials (int32 for INT8, fp32 otherwise), in split order.
 template <int DT>
 __device__ __forceinline__ uint32_t add_acc(uint32_t x, uint32_t y) {
@@ -207,19 +324,24 @@ __device__ __forceinline__ uint32_t add_acc(uint32_t x, uint32_t y) {
 
 template <int N>
 __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N == 8 || N == 16 || N == 32, "tcgen05.ld width");
   if constexpr (N == 32)
     tmem_ld32(taddr, r);
-  else
+  else if constexpr (N == 16)
     tmem_ld16(taddr, r);
+  else
+    tmem_ld8(taddr, r);
 }
 
 template <int DT, int IMG, int BN, int OUT, int XKB>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(cta_threads(OUT), 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                 const __grid_constant__ CUtensorMap tmW, const SpmmArgs a) {
   using C = Cfg<DT, IMG, BN, OUT, XKB>;
   constexpr bool XS = C::XS;
   constexpr bool SP = C::SP;
+  constexpr bool EPI = (OUT & kOutEpi) != 0;
+  static_assert(!EPI || !C::TS, "the runtime output stage stores directly");
   constexpr int KIND = DT == DT_I8 ? 0 : 1;
 
   extern __shared__ uint8_t smem_raw[];
@@ -246,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accf_bar[i], 1);
-      mbar_init(&acce_bar[i], kEpiWarps);
+      mbar_init(&acce_bar[i], C::EPI_WARPS);
     }
     mbar_init(&drain_bar, 1);
     mbar_init(&xfull_bar, 1);
@@ -434,10 +556,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     using OutT = decltype(convert_out<(OUT & 3)>(0u, 1.0f, false));
-    const int ep_tid = threadIdx.x - 64;  // 0 .. 32*kEpiWarps-1
-    const int ew = warp - 2;              // epilogue warp 0..7
+    const int ep_tid = threadIdx.x - 64;  // 0 .. 32*EPI_WARPS-1
+    const int ew = warp - 2;              // epilogue warp 0..EPI_WARPS-1
     const int lq = warp & 3;              // TMEM lane quarter this warp may access
-    const int half = ew >> 2;             // which half of the token columns
+    const int part = ew >> 2;             // which BN/epw slice of the token columns
     uint8_t* stage_buf =
         smem + (size_t)C::STAGES * C::STAGE + C::X_BYTES + (size_t)ew * C::EPI_NB * C::EPI_BUF;
     int buf = 0, acc = 0;
@@ -455,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ep_ok_sh[iter & 1] = got ? 1 : 0;
         NM_TR(TR_E_START, iter);
       }
-      named_bar_sync(1, 32 * kEpiWarps);
+      named_bar_sync(1, 32 * C::EPI_WARPS);
       if (!ep_ok_sh[iter & 1]) break;
       tc_fence_after();
       const int ch0 = w.ct * kRows + lq * 32;  // first channel of this warp's lane quarter
@@ -463,7 +585,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ch_ok = ch < a.n_out;
       const bool has_scale = a.scale != nullptr;
       const float s = (has_scale && ch_ok) ? __ldg(a.scale + ch) : 1.0f;
-      const int col0 = half * C::HALF;         // first token column of this warp within the tile
+      const float bch = (EPI && a.bias && ch_ok) ? __ldg(a.bias + ch) : 0.0f;
+      const int col0 = part * C::WCOLS;        // first token column of this warp within the tile
       const int t0 = w.tt * BN + col0;
       const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(acc * BN + col0);
       if (a.splits == 1) {
@@ -494,15 +617,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (C::EPI_NB == 2) buf ^= 1;
           } else if (ch_ok) {
-            OutT* yp = reinterpret_cast<OutT*>(a.Y) + (size_t)tc0 * a.n_out + ch;
-            const int nvalid = a.T - tc0;
-            if (nvalid >= C::CH) {
-#pragma unroll
-              for (int j = 0; j < C::CH; ++j) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+            if constexpr (EPI) {
+              epi_run<DT, C::CH>(a, EpiCh{s, bch}, r, (size_t)tc0 * a.n_out + ch, a.T - tc0);
             } else {
+              OutT* yp = reinterpret_cast<OutT*>(a.Y) + (size_t)tc0 * a.n_out + ch;
+              const int nvalid = a.T - tc0;
+              if (nvalid >= C::CH) {
 #pragma unroll
-              for (int j = 0; j < C::CH; ++j)
-                if (j < nvalid) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+                for (int j = 0; j < C::CH; ++j) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+              } else {
+#pragma unroll
+                for (int j = 0; j < C::CH; ++j)
+                  if (j < nvalid) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+              }
             }
           }
         }
@@ -524,16 +651,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce_bar[acc]);
         __threadfence();
-        named_bar_sync(1, 32 * kEpiWarps);
+        named_bar_sync(1, 32 * C::EPI_WARPS);
         if (ep_tid == 0) last_sh = (atomicAdd(a.cnt + w.tile, 1) == a.splits - 1);
-        named_bar_sync(1, 32 * kEpiWarps);
+        named_bar_sync(1, 32 * C::EPI_WARPS);
         if (last_sh) {
           __threadfence();
           const uint32_t* tile_base = part + (size_t)w.tile * a.splits * tile_elems;
           // eight columns at a time, every split's loads in flight before any add
-          constexpr int RC = C::HALF < 8 ? C::HALF : 8;
+          constexpr int RC = C::WCOLS < 8 ? C::WCOLS : 8;
 #pragma unroll 1
-          for (int cb = col0; cb < col0 + C::HALF; cb += RC) {
+          for (int cb = col0; cb < col0 + C::WCOLS; cb += RC) {
             uint32_t sum[RC];
             const uint32_t* src = tile_base + (size_t)cb * kRows + lq * 32 + lane;
 #pragma unroll
@@ -548,7 +675,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < RC; ++q) {
               const int t = w.tt * BN + cb + q;
-              if (ch_ok && t < a.T) store_out<(OUT & 3)>(a.Y, (size_t)t * a.n_out + ch, sum[q], s, has_scale);
+              if (ch_ok && t < a.T) {
+                if constexpr (EPI)
+                  epi_one<DT>(a, EpiCh{s, bch}, (size_t)t * a.n_out + ch, sum[q]);
+                else
+                  store_out<(OUT & 3)>(a.Y, (size_t)t * a.n_out + ch, sum[q], s, has_scale);
+              }
             }
           }
           if (ep_tid == 0) a.cnt[w.tile] = 0;  // re-arm for the next launch
@@ -594,14 +726,16 @@ struct PairCfg {
   static constexpr int E_COL0 = 2 * BN;
   static constexpr int COLS_NEEDED = 2 * BN + 2 * E_COLS;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 256 ? 256 : 512;
-  static constexpr int HALF = BN / 2;               // token columns per epilogue warp
-  static constexpr int CH = (HALF % 32 == 0) ? 32 : 16;
-  static constexpr int NCH = HALF / CH;
+  static constexpr int EPI_WARPS = epi_warps(OUT);
+  static constexpr int THREADS = cta_threads(OUT);
+  static constexpr int WCOLS = BN / (EPI_WARPS / 4);  // token columns per epilogue warp
+  static constexpr int CH = (WCOLS % 32 == 0) ? 32 : (WCOLS % 16 == 0) ? 16 : 8;
+  static constexpr int NCH = WCOLS / CH;
   static constexpr int OES = out_bytes(OUT);
   static constexpr int EPI_BUF = CH * 32 * OES;
   static constexpr bool TS = (OUT & kOutDirect) == 0;
-  static constexpr int EPI_NB = (kSmemBudget - 2 * kEpiWarps * EPI_BUF) / STAGE >= 4 ? 2 : 1;
-  static constexpr int EPI_BYTES = TS ? EPI_NB * kEpiWarps * EPI_BUF : 0;
+  static constexpr int EPI_NB = (kSmemBudget - 2 * EPI_WARPS * EPI_BUF) / STAGE >= 4 ? 2 : 1;
+  static constexpr int EPI_BYTES = TS ? EPI_NB * EPI_WARPS * EPI_BUF : 0;
   static constexpr int STAGES_FIT = (kSmemBudget - EPI_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int SMEM = STAGES * STAGE + EPI_BYTES + 1024;
@@ -609,15 +743,17 @@ struct PairCfg {
   static_assert(STAGES >= 2, "need at least two stages");
   static_assert(COLS_NEEDED <= 512, "tensor memory overflow");
   static_assert(BN % 32 == 0 && BN <= 256, "pair MMA N");
-  static_assert(HALF % CH == 0, "epilogue chunking");
+  static_assert(WCOLS % CH == 0, "epilogue chunking");
 };
 
 template <int DT, int IMG, int BN, int OUT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
     spmm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                      const __grid_constant__ CUtensorMap tmW, const SpmmArgs a) {
   using C = PairCfg<DT, IMG, BN, OUT>;
   constexpr bool SP = C::SP;
+  constexpr bool EPI = (OUT & kOutEpi) != 0;
+  static_assert(!EPI || !C::TS, "the runtime output stage stores directly");
   constexpr int KIND = DT == DT_I8 ? 0 : 1;
 
   extern __shared__ uint8_t smem_raw[];
@@ -643,7 +779,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accf_bar[i], 1);
-      mbar_init(&acce_bar[i], 2 * kEpiWarps);  // both CTAs' epilogue warps release the leader's accumulator
+      mbar_init(&acce_bar[i], 2 * C::EPI_WARPS);  // both CTAs' epilogue warps release the leader's accumulator
     }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -799,7 +935,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int ep_tid = threadIdx.x - 64;
     const int ew = warp - 2;
     const int lq = warp & 3;
-    const int half = ew >> 2;
+    const int part = ew >> 2;
     uint8_t* stage_buf = smem + (size_t)C::STAGES * C::STAGE + (size_t)ew * C::EPI_NB * C::EPI_BUF;
     int buf = 0, acc = 0, iter = 0;
     uint32_t acc_phase = 0;
@@ -812,7 +948,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ep_ok_sh[iter & 1] = got ? 1 : 0;
         NM_TR(TR_E_START, iter);
       }
-      named_bar_sync(1, 32 * kEpiWarps);
+      named_bar_sync(1, 32 * C::EPI_WARPS);
       if (!ep_ok_sh[iter & 1]) break;
       tc_fence_after();
       const int ch0 = ct * kRows + lq * 32;
@@ -820,7 +956,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool ch_ok = ch < a.n_out;
       const bool has_scale = a.scale != nullptr;
       const float s = (has_scale && ch_ok) ? __ldg(a.scale + ch) : 1.0f;
-      const int col0 = half * C::HALF;
+      const float bch = (EPI && a.bias && ch_ok) ? __ldg(a.bias + ch) : 0.0f;
+      const int col0 = part * C::WCOLS;
       const int t0 = tt * BN + col0;
       const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(acc * BN + col0);
 #pragma unroll 1
@@ -855,15 +992,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if (C::EPI_NB == 2) buf ^= 1;
         } else if (ch_ok) {
-          OutT* yp = reinterpret_cast<OutT*>(a.Y) + (size_t)tc0 * a.n_out + ch;
-          const int nvalid = a.T - tc0;
-          if (nvalid >= C::CH) {
-#pragma unroll
-            for (int j = 0; j < C::CH; ++j) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+          if constexpr (EPI) {
+            epi_run<DT, C::CH>(a, EpiCh{s, bch}, r, (size_t)tc0 * a.n_out + ch, a.T - tc0);
           } else {
+            OutT* yp = reinterpret_cast<OutT*>(a.Y) + (size_t)tc0 * a.n_out + ch;
+            const int nvalid = a.T - tc0;
+            if (nvalid >= C::CH) {
 #pragma unroll
-            for (int j = 0; j < C::CH; ++j)
-              if (j < nvalid) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+              for (int j = 0; j < C::CH; ++j) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::CH; ++j)
+                if (j < nvalid) yp[(size_t)j * a.n_out] = convert_out<(OUT & 3)>(r[j], s, has_scale);
+            }
           }
         }
       }
@@ -892,11 +1033,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // Launch with programmatic stream serialization, so the kernel's prologue can
 // overlap the tail of the previous kernel in the stream (see pdl_wait).
 template <typename Kern>
-static cudaError_t launch_pdl(Kern kern, dim3 grid, int smem, cudaStream_t s, const CUtensorMap& tmX,
+static cudaError_t launch_pdl(Kern kern, dim3 grid, int threads, int smem, cudaStream_t s, const CUtensorMap& tmX,
                               const CUtensorMap& tmY, const CUtensorMap& tmW, const SpmmArgs& a) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = s;
   cudaLaunchAttribute attr;
@@ -918,7 +1059,7 @@ static cudaError_t launch_t(const CUtensorMap* tmX, const CUtensorMap* tmY, cons
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(kern, dim3(p.grid), C::SMEM, s, *tmX, *tmY, *tmW, a);
+  return launch_pdl(kern, dim3(p.grid), C::THREADS, C::SMEM, s, *tmX, *tmY, *tmW, a);
 }
 
 template <int DT, int IMG, int BN, int OUT>
@@ -932,7 +1073,7 @@ static cudaError_t launch_pair_t(const CUtensorMap* tmX, const CUtensorMap* tmY,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(kern, dim3(2 * p.grid), C::SMEM, s, *tmX, *tmY, *tmW, a);  // p.grid = CTA pairs
+  return launch_pdl(kern, dim3(2 * p.grid), C::THREADS, C::SMEM, s, *tmX, *tmY, *tmW, a);  // p.grid = CTA pairs
 }
 
 int pair_max_clusters(int dt, int img, int bn, int out);
@@ -973,6 +1114,17 @@ template <int OUT_TS>
 static cudaError_t launch_dt(const nm_handle* h, const CUtensorMap* tmX, const CUtensorMap* tmY,
                              const CUtensorMap* tmW, const Plan& p, const SpmmArgs& a, cudaStream_t s) {
   constexpr int D = OUT_TS;  // 0 or kOutDirect
+  if constexpr (D == kOutDirect) {
+    if (a.out_ty >= 0) {  // runtime output stage
+      switch (h->dt) {
+        case DT_I8: return launch_img<DT_I8, kOutEpi | kOutDirect>(h->img, tmX, tmY, tmW, p, a, s);
+        case DT_F16: return launch_img<DT_F16, kOutEpi | kOutDirect>(h->img, tmX, tmY, tmW, p, a, s);
+        default: return launch_img<DT_BF16, kOutEpi | kOutDirect>(h->img, tmX, tmY, tmW, p, a, s);
+      }
+    }
+  } else {
+    if (a.out_ty >= 0) return cudaErrorInvalidValue;  // the runtime output stage stores directly
+  }
   switch (h->dt) {
     case DT_I8:
       return a.scale ? launch_img<DT_I8, OUT_F32 | D>(h->img, tmX, tmY, tmW, p, a, s)
@@ -998,7 +1150,7 @@ static int max_clusters_t() {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.attrs = nullptr;  // the kernel declares its cluster shape (2 CTAs) at compile time
     cfg.numAttrs = 0;

@@ -39,6 +39,11 @@ def float_normal(shape, std: float, seed: int, dtype: str) -> torch.Tensor:
     return t.to(torch.float16 if dtype == FP16 else torch.bfloat16)
 
 
+def normal_f32(shape, std: float, seed: int) -> torch.Tensor:
+    """fp32 N(0, std^2) (per-channel biases of the fused output stage)."""
+    return torch.randn(tuple(shape), generator=_gen(seed), dtype=torch.float32) * std
+
+
 def scale_uniform(n: int, lo: float, hi: float, seed: int) -> torch.Tensor:
     """Per-output-channel fp32 scale, uniform on [lo, hi)."""
     return torch.rand((n,), generator=_gen(seed), dtype=torch.float32) * (hi - lo) + lo
