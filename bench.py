@@ -244,6 +244,51 @@ def alg_bytes_any(l, out_es: int | None = None, biased: bool = False) -> int:
             + (4 * l.n_out if biased else 0))
 
 
+def run_lut(args) -> None:
+    """Calibrated LUT latency predictor on the 48 ViT-B linears: profile every
+    (shape, pattern) at T = 197 and 50432, calibrate on random layer-wise
+    assignments, then report the prediction error on held-out assignments and
+    on the mixed sequence (seed 5), each against its measured latency."""
+    from structured_sparse_gemm_compress_b200 import lut
+
+    torch.cuda.set_device(0)
+    layers = lut.vit_b_layers()
+    shapes = sorted({(l.K, l.n_out) for l in layers})
+    Ts = [197, 50432]
+    ws = lut._Workspace()
+    t0 = time.time()
+    L = lut.profile(shapes, list(lut.PATTERNS), Ts, reps=20, ws=ws)
+    t_prof = time.time() - t0
+    calib = []
+    for T in Ts:
+        for i in range(4):
+            asg = lut.random_assignment(len(layers), 100 + i)
+            calib.append((layers, asg, T, lut.measure_sequence(layers, asg, T, reps=3, ws=ws)))
+    L.calibrate(calib)
+    mixed = [("dense" if l.N == l.M else l.nm) for l in inputs.vit_b_mixed(197)]
+    per_t, errs = {}, []
+    for T in Ts:
+        rows = []
+        for i, asg in enumerate([lut.random_assignment(len(layers), 200 + i) for i in range(6)] + [mixed]):
+            meas = lut.measure_sequence(layers, asg, T, reps=3, ws=ws)
+            pred = L.predict(layers, asg, T)
+            rows.append({"assignment": "mixed seed 5" if i == 6 else f"random seed {200 + i}",
+                         "measured_us": round(meas, 1), "predicted_us": round(pred, 1),
+                         "raw_lut_sum_us": round(L.raw_sum(layers, asg, T), 1),
+                         "err_pct": round(100 * (pred - meas) / meas, 2)})
+            errs.append(abs(pred - meas) / meas)
+        per_t[str(T)] = rows
+    line = {"config": {"workload": "calibrated LUT latency predictor, 48 ViT-B linears, INT8 + scale, "
+                                   "patterns {dense,4:8,2:4,2:8,1:4}, T in {197, 50432}"},
+            "metric": "mean |predicted - measured| / measured over held-out layer-wise assignments",
+            "value": round(100 * float(np.mean(errs)), 3), "unit": "%", "higher_is_better": False,
+            "max_err_pct": round(100 * float(np.max(errs)), 3),
+            "calibration": {"a": round(L.a, 4), "b_us_per_layer": round(L.b, 3), "samples": len(calib)},
+            "lut_entries": len(L.table), "profile_s": round(t_prof, 1), "per_T": per_t,
+            "data": "synthetic", "dtype": "int8"}
+    print(json.dumps(line), flush=True)
+
+
 def run_config(name: str, args) -> None:
     import structured_sparse_gemm_compress_b200 as nm
 
@@ -386,7 +431,7 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
-    ap.add_argument("--config", default=None, choices=["single", "vitl", "swin", "mixed1", "mixed256", "int8out"],
+    ap.add_argument("--config", default=None, choices=["single", "vitl", "swin", "mixed1", "mixed256", "int8out", "lut"],
                     help="measure another workload (one JSON line) instead of the default ViT-B INT8 set")
     ap.add_argument("--only", action="append", default=[],
                     help="restrict to problems like vitb.fc1/2:4 (profiling a single kernel shape)")
@@ -401,7 +446,7 @@ def main() -> None:
         return
     if args.config is not None:
         if rank == 0:
-            run_config(args.config, args)
+            run_lut(args) if args.config == "lut" else run_config(args.config, args)
         return
 
     import structured_sparse_gemm_compress_b200 as nm

@@ -1,0 +1,215 @@
+"""Calibrated lookup-table (LUT) latency predictor for layer-wise N:M sequences.
+
+"Realizable N:M Sparse Transformer Inference via Search-Kernel Co-Design"
+(arXiv 2607.12505), sections 1 and 3: the layer-wise N:M search relies on a
+calibrated, profiling-based LUT latency predictor that keeps candidate
+configurations inside the deployment latency budget.  The pages give no more
+detail, so this module takes the plainest reading:
+
+* the table holds the measured latency of one ``nm_spmm`` launch for every
+  (K, n_out, pattern, T) profiled on the target GPU; between profiled token
+  counts the latency is interpolated linearly in T (extrapolated from the two
+  nearest points outside the profiled range);
+* a configuration (one pattern per linear layer) is predicted by summing its
+  layers' table entries, then calibrated against measured end-to-end sequence
+  latencies with a least-squares fit  measured ~ a * sum + b * layers  (a
+  absorbs overlap and cache effects between back-to-back launches, b a fixed
+  cost per launch).
+
+Profiling and sequence timing run the product kernels through the package's
+binding; the table logic itself is plain host code.
+"""
+from __future__ import annotations
+
+import json
+import random
+from dataclasses import dataclass
+
+import numpy as np
+
+PATTERNS = {"dense": (4, 4), "4:8": (4, 8), "2:4": (2, 4), "2:8": (2, 8), "1:4": (1, 4)}
+
+
+@dataclass(frozen=True)
+class LayerSpec:
+    """One linear layer: Y[T, n_out] = X[T, K] . W[n_out, K]^T."""
+    name: str
+    K: int
+    n_out: int
+
+
+def vit_b_layers(blocks: int = 12) -> list[LayerSpec]:
+    """The 4 linears of each ViT-B/16 block (qkv, proj, fc1, fc2)."""
+    out = []
+    for b in range(blocks):
+        out += [LayerSpec(f"b{b}.qkv", 768, 2304), LayerSpec(f"b{b}.proj", 768, 768),
+                LayerSpec(f"b{b}.fc1", 768, 3072), LayerSpec(f"b{b}.fc2", 3072, 768)]
+    return out
+
+
+def random_assignment(n_layers: int, seed: int, patterns=tuple(PATTERNS)) -> list[str]:
+    rng = random.Random(seed)
+    return [rng.choice(patterns) for _ in range(n_layers)]
+
+
+class LatencyLUT:
+    """Measured per-launch latency table plus the sequence calibration."""
+
+    def __init__(self, table: dict[tuple[int, int, str, int], float], meta: dict | None = None,
+                 a: float = 1.0, b: float = 0.0):
+        self.table = dict(table)
+        self.meta = dict(meta or {})
+        self.a, self.b = float(a), float(b)
+
+    # ---------------------------------------------------------------- lookup
+    def lookup(self, K: int, n_out: int, pattern: str, T: int) -> float:
+        """Latency (us) of one launch; linear in T between profiled token counts."""
+        pts = sorted((t, us) for (k, n, p, t), us in self.table.items() if (k, n, p) == (K, n_out, pattern))
+        if not pts:
+            raise KeyError(f"no entry for K={K} n_out={n_out} pattern={pattern}")
+        ts = [t for t, _ in pts]
+        if T in ts:
+            return pts[ts.index(T)][1]
+        if len(pts) == 1:
+            raise KeyError(f"only T={ts[0]} profiled for K={K} n_out={n_out} pattern={pattern}")
+        i = int(np.searchsorted(ts, T))
+        i = min(max(i, 1), len(pts) - 1)   # bracketing pair, or the two nearest at an end
+        (t0, u0), (t1, u1) = pts[i - 1], pts[i]
+        return u0 + (u1 - u0) * (T - t0) / (t1 - t0)
+
+    def raw_sum(self, layers: list[LayerSpec], assignment: list[str], T: int) -> float:
+        if len(layers) != len(assignment):
+            raise ValueError("one pattern per layer")
+        return sum(self.lookup(l.K, l.n_out, p, T) for l, p in zip(layers, assignment))
+
+    def predict(self, layers: list[LayerSpec], assignment: list[str], T: int) -> float:
+        """Calibrated end-to-end latency (us) of the layer sequence."""
+        return self.a * self.raw_sum(layers, assignment, T) + self.b * len(layers)
+
+    # ---------------------------------------------------------------- calibration
+    def calibrate(self, samples: list[tuple[list[LayerSpec], list[str], int, float]]) -> tuple[float, float]:
+        """Least-squares fit of measured ~ a * raw_sum + b * n_layers over
+        (layers, assignment, T, measured_us) samples; sets and returns (a, b)."""
+        A = np.array([[self.raw_sum(ls, asg, T), float(len(ls))] for ls, asg, T, _ in samples])
+        y = np.array([m for *_, m in samples])
+        if len(samples) >= 2 and np.linalg.matrix_rank(A) == 2:
+            sol, *_ = np.linalg.lstsq(A, y, rcond=None)
+            self.a, self.b = float(sol[0]), float(sol[1])
+        else:  # one sample (or all with the same layer count and sum): scale only
+            self.a, self.b = float(y.sum() / A[:, 0].sum()), 0.0
+        return self.a, self.b
+
+    # ---------------------------------------------------------------- persistence
+    def to_json(self) -> str:
+        rows = [{"K": k, "n_out": n, "pattern": p, "T": t, "us": us} for (k, n, p, t), us in sorted(self.table.items())]
+        return json.dumps({"meta": self.meta, "calibration": {"a": self.a, "b": self.b}, "entries": rows}, indent=1)
+
+    @staticmethod
+    def from_json(text: str) -> "LatencyLUT":
+        d = json.loads(text)
+        table = {(r["K"], r["n_out"], r["pattern"], r["T"]): float(r["us"]) for r in d["entries"]}
+        cal = d.get("calibration", {})
+        return LatencyLUT(table, d.get("meta"), cal.get("a", 1.0), cal.get("b", 0.0))
+
+
+# -------------------------------------------------------------------- GPU side
+
+def _graph_time_us(launch, reps: int) -> float:
+    """Average time (us) of one call of ``launch(stream)`` over ``reps`` calls
+    captured back to back in one CUDA graph, after warm-up; events only around
+    the whole replay."""
+    import torch
+
+    for _ in range(3):
+        launch(None)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+        for _ in range(reps):
+            launch(cap)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / reps
+    del g
+    return us
+
+
+class _Workspace:
+    """Seeded device operands per (K, n_out) and per T, reused across patterns."""
+
+    def __init__(self, seed: int = 11):
+        self.seed = seed
+        self.W, self.X, self.s = {}, {}, {}
+
+    def weight(self, K, n_out):
+        import torch
+
+        from . import inputs
+        if (K, n_out) not in self.W:
+            self.W[(K, n_out)] = inputs.int8_uniform((n_out, K), -127, 127, self.seed + K + n_out).cuda()
+            self.s[(K, n_out)] = inputs.scale_uniform(n_out, 0.001, 0.01, self.seed + 2 * K + n_out).cuda()
+        return self.W[(K, n_out)], self.s[(K, n_out)]
+
+    def act(self, T, K):
+        from . import inputs
+        if (T, K) not in self.X:
+            self.X[(T, K)] = inputs.int8_uniform((T, K), -128, 127, self.seed + T + K).cuda()
+        return self.X[(T, K)]
+
+
+def profile(shapes: list[tuple[int, int]], patterns: list[str], Ts: list[int], reps: int = 20,
+            ws: _Workspace | None = None) -> LatencyLUT:
+    """Profile ``nm_spmm`` (INT8, per-channel scale, fp32 output) for every
+    (K, n_out) in ``shapes``, pattern and token count on the current GPU."""
+    import torch
+
+    import structured_sparse_gemm_compress_b200 as nm
+
+    ws = ws or _Workspace()
+    table = {}
+    for K, n_out in shapes:
+        W, s = ws.weight(K, n_out)
+        for p in patterns:
+            N, M = PATTERNS[p]
+            h = nm.nm_compress(W, N, M)
+            for T in Ts:
+                X = ws.act(T, K)
+                Y = torch.empty((T, n_out), dtype=torch.float32, device="cuda")
+                table[(K, n_out, p, T)] = _graph_time_us(
+                    lambda st, h=h, X=X, Y=Y: nm.nm_spmm(h, X, Y=Y, scale=s, stream=st), reps)
+            h.destroy()
+    meta = {"device": torch.cuda.get_device_name(), "reps": reps, "dtype": "int8", "output": "fp32 scaled"}
+    return LatencyLUT(table, meta)
+
+
+def measure_sequence(layers: list[LayerSpec], assignment: list[str], T: int, reps: int = 5,
+                     ws: _Workspace | None = None) -> float:
+    """Measured latency (us) of the whole layer sequence, launched back to back
+    in one stream (one CUDA graph of ``reps`` passes, events around it)."""
+    import torch
+
+    import structured_sparse_gemm_compress_b200 as nm
+
+    ws = ws or _Workspace()
+    handles, Ys = [], []
+    for l, p in zip(layers, assignment):
+        W, s = ws.weight(l.K, l.n_out)
+        N, M = PATTERNS[p]
+        handles.append((nm.nm_compress(W, N, M), ws.act(T, l.K), s))
+        Ys.append(torch.empty((T, l.n_out), dtype=torch.float32, device="cuda"))
+
+    def one_pass(st):
+        for (h, X, s), Y in zip(handles, Ys):
+            nm.nm_spmm(h, X, Y=Y, scale=s, stream=st)
+
+    us = _graph_time_us(one_pass, reps)
+    for h, _, _ in handles:
+        h.destroy()
+    return us
