@@ -229,13 +229,22 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
     p.grid = std::min(p.units, sms);
     return p;
   }
-  const int bns[3] = {128, 64, 32};
+  // Streaming token tile: minimise (waves of persistent CTAs) x (cost of one
+  // tile).  Measured on B200 (ViT-B INT8 shapes at T = 12608 and 50432): a tile
+  // costs about (BN + 140) token columns' worth -- its fixed part (weight chunk
+  // loads, MMA issue per stage, epilogue start) equals ~140 columns -- and 18 %
+  // more when only three pipeline stages fit in shared memory.  Tiles that
+  // would leave two stages are not used.
+  const int bns[4] = {192, 128, 64, 32};
   double best = 1e300;
   for (int bn : bns) {
     if (forced_bn && bn != forced_bn) continue;
+    const int stage = nm::chunk_bytes(h->dt, h->img) + bn * 256;  // packed chunk + 256 B of X per token
+    const int stages = std::min(8, (227 * 1024 - 1024) / stage);
+    if (stages < 3 && bn > 128) continue;
     const int64_t tiles = (int64_t)h->n_ct * ((T + bn - 1) / bn);
     const int64_t waves = (tiles + sms - 1) / sms;
-    const double cost = (double)waves * (bn + 32);
+    const double cost = (double)waves * (bn + 140) * (stages >= 4 ? 1.0 : 1.18);
     if (cost < best) {
       best = cost;
       p.bn = bn;

@@ -80,7 +80,7 @@ struct Cfg {
   static constexpr int EPI_WARPS = epi_warps(OUT);
   static constexpr int THREADS = cta_threads(OUT);
   static constexpr int WCOLS = BN / (EPI_WARPS / 4);
-  static constexpr int CH = WCOLS >= 32 ? 32 : WCOLS;
+  static constexpr int CH = (WCOLS % 32 == 0) ? 32 : (WCOLS % 16 == 0) ? 16 : 8;
   static constexpr int NCH = WCOLS / CH;
   static constexpr int OES = out_bytes(OUT);
   static constexpr int EPI_BUF = CH * 32 * OES;     // one staged [CH tokens][32 channels] tile
@@ -1099,6 +1099,7 @@ static cudaError_t launch_bn(const CUtensorMap* tmX, const CUtensorMap* tmY, con
     case 32: return launch_t<DT, IMG, 32, OUT, 0>(tmX, tmY, tmW, p, a, s);
     case 64: return launch_t<DT, IMG, 64, OUT, 0>(tmX, tmY, tmW, p, a, s);
     case 128: return launch_t<DT, IMG, 128, OUT, 0>(tmX, tmY, tmW, p, a, s);
+    case 192: return launch_t<DT, IMG, 192, OUT, 0>(tmX, tmY, tmW, p, a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -145,7 +145,7 @@ def test_float_handles_output_stage(dtype, out, act):
 
 
 @pytest.mark.parametrize("plan", [
-    {"NMSPMM_FORCE_BN": "32"}, {"NMSPMM_FORCE_BN": "64"}, {"NMSPMM_FORCE_SPLITK": "3"},
+    {"NMSPMM_FORCE_BN": "32"}, {"NMSPMM_FORCE_BN": "64"}, {"NMSPMM_FORCE_BN": "192"}, {"NMSPMM_FORCE_SPLITK": "3"},
     {"NMSPMM_FORCE_XS": "1"}, {"NMSPMM_FORCE_PAIR": "1"}, {"NMSPMM_FORCE_PAIR": "1", "NMSPMM_FORCE_BN": "224"},
     {"NMSPMM_FORCE_GRID": "5"}], ids=lambda d: ",".join(f"{k[13:]}={v}" for k, v in d.items()))
 @pytest.mark.parametrize("out", ["int8", "bfloat16"])

@@ -158,7 +158,7 @@ def test_spmm_fp16_scaled():
     _assert_float_close(Y, ref, "fp16")
 
 
-@pytest.mark.parametrize("bn", ["32", "64", "128"])
+@pytest.mark.parametrize("bn", ["32", "64", "128", "192"])
 @pytest.mark.parametrize("split", ["1", "2", "3", "5"])
 def test_forced_tiles_and_splits_are_bit_identical(monkeypatch, bn, split):
     """Adaptive parallelism must not change INT8 results at all."""
@@ -254,6 +254,18 @@ def test_forced_split_fp16_within_tolerance(monkeypatch, split):
     h = nm.nm_compress(W.cuda(), 2, 8)
     Y = nm.nm_spmm(h, X.cuda())
     _assert_float_close(Y, oracle.spmm(_np(X, "fp16"), _np(W, "fp16"), 2, 8, dtype="fp16"), "fp16")
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("bn", ["64", "192"])
+def test_forced_tile_float_within_tolerance(monkeypatch, dtype, bn):
+    W = _weights(dtype, 300, 1024, seed=61)
+    X = _acts(dtype, 700, 1024, seed=62)
+    monkeypatch.setenv("NMSPMM_FORCE_BN", bn)
+    monkeypatch.setenv("NMSPMM_FORCE_PAIR", "0")
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    Y = nm.nm_spmm(h, X.cuda())
+    _assert_float_close(Y, oracle.spmm(_np(X, dtype), _np(W, dtype), 2, 4, dtype=dtype), dtype)
 
 
 # --------------------------------------------------------------------------- full-size workloads (sampled)
