@@ -166,16 +166,13 @@ void out_type(const nm_handle* h, bool scaled, int* es, int* ty) {
   }
 }
 
-// Adaptive parallelism: pick the token tile and split-K factor for this shape.
-// Token tile: minimise (waves of persistent CTAs) x (per-tile cost ~ bn + 32).
-// Split-K: only when even the smallest tile leaves most SMs idle; partials are
-// reduced by the last-arriving CTA, so the reduction costs one extra pass over
-// the tile per split, which is why splits stay bounded by the idle SMs.
 int out_code(const nm_handle* h, bool scaled) {
   if (h->dt == nm::DT_I8) return scaled ? nm::OUT_F32 : nm::OUT_I32;
   return h->dt == nm::DT_F16 ? nm::OUT_F16 : nm::OUT_BF16;
 }
 
+// Adaptive parallelism: pick the kernel (CTA pair or single SM), the token tile
+// and the split-K factor for this shape (rules and their measurements below).
 nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
   nm::Plan p;
   const int forced_bn = env_int("NMSPMM_FORCE_BN", 0);
@@ -255,9 +252,12 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
   int splits = 1;
   if (forced_split > 0) {
     splits = forced_split;
-  } else if (tiles * 2 <= sms && h->n_kb >= 2) {
-    splits = (int)std::min<int64_t>(h->n_kb, sms / tiles);
   }
+  // No split-K by default: measured on B200, the partial round trip (write,
+  // arrival counter, last-arriver reduction) costs more than the idle SMs it
+  // fills, down to 6 tiles on 148 SMs (ViT-B qkv/proj/fc1 at T = 16, 64, 197:
+  // 3.7-3.8 us unsplit against 5.8-13 us split; fc2 at T = 64: 6.9 vs 8.3 us).
+  // The split-K path stays available (NMSPMM_FORCE_SPLITK) and tested.
   splits = std::max(1, std::min(splits, h->n_kb));
   p.kb_per_split = (h->n_kb + splits - 1) / splits;
   p.splits = (h->n_kb + p.kb_per_split - 1) / p.kb_per_split;  // every split owns >= 1 k-block
