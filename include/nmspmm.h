@@ -64,7 +64,9 @@ typedef struct nm_handle nm_handle;
  *         stream has passed this call.
  * (N, M)  one of (1,4), (2,4), (2,8), (4,8), or N == M with M in {4, 8}
  *         (dense pass-through).  Other pairs -> NM_ERR_UNSUPPORTED.
- * k       multiple of M (else NM_ERR_INVALID); n_out, k > 0, at most 2^24.
+ * k       multiple of M (else NM_ERR_INVALID); n_out, k > 0, at most 2^24;
+ *         for NM_INT8 k at most 2^17 (so that k * 128 * 127 fits the int32
+ *         accumulator exactly), else NM_ERR_UNSUPPORTED.
  * out     receives the handle; *out is NULL on failure.
  * Allocates device memory (NM_ERR_OOM on failure); returns without waiting
  * for the kernels.

@@ -422,6 +422,9 @@ nm_status nm_compress(const void* W_dev, int64_t n_out, int64_t k, nm_dtype dt, 
   if ((int)dt < 0 || (int)dt > 2) return fail(NM_ERR_INVALID, "unknown dtype %d", (int)dt);
   if (n_out <= 0 || k <= 0) return fail(NM_ERR_INVALID, "n_out and k must be positive");
   if (n_out > (1 << 24) || k > (1 << 24)) return fail(NM_ERR_UNSUPPORTED, "n_out and k are limited to 2^24");
+  // INT8 accumulates exactly in int32: |acc| <= k * 128 * 127 must stay below 2^31.
+  if (dt == NM_INT8 && k > (1 << 17))
+    return fail(NM_ERR_UNSUPPORTED, "INT8 k is limited to 2^17 (int32 accumulation must not overflow)");
   if (M <= 0 || N <= 0 || N > M) return fail(NM_ERR_INVALID, "bad N:M %d:%d", N, M);
   const bool sp24 = (N == 1 && M == 4) || (N == 2 && M == 4) || (N == 2 && M == 8);
   const bool dense = (N == 4 && M == 8) || (N == M && (M == 4 || M == 8));

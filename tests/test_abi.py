@@ -53,6 +53,7 @@ def _compress_raw(W_ptr, n_out, k, dt, N, M):
     ((16, 4, 10, nm.NM_INT8, 2, 4), nm.NM_ERR_INVALID),           # k % M != 0
     ((17, 4, 8, nm.NM_FP16, 2, 4), nm.NM_ERR_INVALID),            # misaligned fp16 W
     ((16, 1 << 25, 8, nm.NM_INT8, 2, 4), nm.NM_ERR_UNSUPPORTED),  # n_out above 2^24
+    ((16, 4, (1 << 17) + 4, nm.NM_INT8, 2, 4), nm.NM_ERR_UNSUPPORTED),  # INT8 k: int32 could overflow
 ])
 def test_compress_rejects_before_touching_the_device(args, status):
     st, handle = _compress_raw(*args)

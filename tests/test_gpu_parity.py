@@ -335,6 +335,35 @@ def test_vit_b_mixed_sequence(T):
 # --------------------------------------------------------------------------- edge cases and errors
 
 
+@pytest.mark.parametrize("N,M", [(2, 4), (4, 8), (8, 8)])
+def test_extreme_values_bit_exact(N, M):
+    """Largest accumulator magnitudes: X = -128 everywhere, W at +-127 (and
+    ties everywhere, so the tie rule decides every kept position)."""
+    n_out, K, T = 256, 4096, 130
+    sign = torch.where(inputs.int8_uniform((n_out, K), 0, 1, seed=71) > 0, 127, -127).to(torch.int8)
+    sign[:8] = 127    # rows whose every kept product is -128 * 127
+    sign[8:16] = -127
+    X = torch.full((T, K), -128, dtype=torch.int8)
+    h = nm.nm_compress(sign.cuda(), N, M)
+    Y = nm.nm_spmm(h, X.cuda())
+    ref = oracle.spmm(X.numpy(), sign.numpy(), N, M)
+    assert np.abs(ref).max() == 128 * 127 * K * N // M  # the largest magnitude the shape allows
+    assert np.array_equal(Y.cpu().numpy(), ref)
+
+
+def test_long_k_and_many_channel_tiles():
+    """K = 16384 (64 k-blocks, CTA-pair kernel) and n_out = 20000 (157 channel
+    tiles, more than the SMs), ragged in both."""
+    for (T, n_out, K, seed) in ((130, 200, 16384, 81), (70, 20000, 256, 82)):
+        W = _weights("int8", n_out, K, seed=seed)
+        X = _acts("int8", T, K, seed=seed + 1)
+        s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=seed + 2)
+        h = nm.nm_compress(W.cuda(), 2, 4)
+        Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
+        ref = oracle.spmm(X.numpy(), W.numpy(), 2, 4, scale=s.numpy())
+        assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
 def test_t_zero_is_noop():
     h = nm.nm_compress(_weights("int8", 64, 64, 1).cuda(), 2, 4)
     X = torch.empty((0, 64), dtype=torch.int8, device="cuda")
