@@ -83,9 +83,11 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms while running;
+    the summary keeps the samples taken inside the window marked by
+    ``mark_start``/``mark_end`` (the timed region)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -93,6 +95,13 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -100,7 +109,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.proc = None
         time.sleep(0.3)
@@ -116,22 +125,35 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self) -> dict:
+        import datetime
+
         rows = []
         if self.path and os.path.exists(self.path):
             for line in open(self.path):
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
+                if len(parts) >= 10:
                     rows.append(parts)
             os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        inside = []
+        if self.t0 is not None and self.t1 is not None:
+            for r in rows:
+                try:
+                    ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    continue
+                if self.t0 <= ts <= self.t1:
+                    inside.append(r)
+        window = len(inside)
+        rows = [r[1:] for r in (inside or rows)]
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         busy = [s for s in sm if s > 0.5 * max(mx or [1])] or sm
         return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "samples_in_timed_region": window}
 
 
 # --------------------------------------------------------------------------- multi-rank plumbing
@@ -480,7 +502,7 @@ def run_config(name: str, args) -> None:
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nm", choices=["nm", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=None)
@@ -566,35 +588,43 @@ def main() -> None:
         if nm.nm_device_status(h) != nm.NM_OK:
             raise RuntimeError(nm.nm_last_error())
 
-    # The K timed steps: captured once into a CUDA graph (one launch for the whole
-    # region; consecutive SpMMs overlap launch and prologue through programmatic
-    # dependent launch), replayed once untimed and once timed.  No event is
-    # recorded inside the region: an event node between two kernels of a graph
-    # serialises them and costs more than a short kernel.  --no-graph runs the
-    # steps eagerly.
-    graph = None
+    # The K timed steps: CUDA graphs of up to 50 steps each (consecutive SpMMs
+    # overlap launch and prologue through programmatic dependent launch),
+    # replayed back to back so that exactly K steps run in the timed region,
+    # after one untimed pass.  No event is recorded inside a graph: an event node
+    # between two kernels serialises them and costs more than a short kernel.
+    # --no-graph runs the steps eagerly.
+    graphs, built = [], {}
     if not args.no_graph:
-        graph = torch.cuda.CUDAGraph()
-        cap, cap_pack = torch.cuda.Stream(), torch.cuda.Stream()
-        cap.wait_stream(stream)
-        with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
-            for k in range(args.steps):
-                step(st=cap, ps=cap_pack)
-        graph.replay()  # upload + one untimed pass
+        chunk = min(args.steps, 50)
+        sizes = [chunk] * (args.steps // chunk) + ([args.steps % chunk] if args.steps % chunk else [])
+        for n in sorted(set(sizes)):
+            g = torch.cuda.CUDAGraph()
+            cap, cap_pack = torch.cuda.Stream(), torch.cuda.Stream()
+            cap.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+                for k in range(n):
+                    step(st=cap, ps=cap_pack)
+            g.replay()  # upload + one untimed pass
+            built[n] = g
+        graphs = [built[n] for n in sizes]
         torch.cuda.synchronize()
 
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         barrier()
         torch.cuda.synchronize()
+        clk.mark_start()
         start.record(stream)
-        if graph is not None:
-            graph.replay()
+        if graphs:
+            for g in graphs:
+                g.replay()
         else:
             for k in range(args.steps):
                 step()
         stop.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
         barrier()
     ms_local = start.elapsed_time(stop)
     ms = max_over_ranks(ms_local, dist, dev)
@@ -719,7 +749,7 @@ def main() -> None:
                "sample": f"first {rows} of 12608 tokens of each of the 16 (layer, N:M) problems "
                          f"(compress + decompress + triple-loop GEMM), {secs:.1f} s"}
 
-    del graph
+    del graphs, built
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
@@ -733,7 +763,7 @@ def main() -> None:
                    "global_batch_tokens": 12608 * world, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2: each step streams ~1.7 GB",
                    "step": "per (layer, N:M): nm_recompress + nm_spmm",
-                   "launch": "eager" if args.no_graph else "cuda-graph of the K timed steps"},
+                   "launch": "eager" if args.no_graph else "CUDA graphs of up to 50 steps replayed back to back"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
                      "kernel": "nm_spmm kernels (streaming and CTA-pair variants): average launch = timed region / (16 K) launches on its stream", "peak_source": pk["source"]},
