@@ -36,6 +36,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <atomic>
 #include <type_traits>
 
 namespace nm {
@@ -1048,17 +1049,28 @@ static cudaError_t launch_pdl(Kern kern, dim3 grid, int threads, int smem, cudaS
   return cudaLaunchKernelEx(&cfg, kern, tmX, tmY, tmW, a);
 }
 
+// The dynamic shared-memory opt-in is a per-device property of a kernel: set it
+// once per (kernel, device), remembered in a bit mask of device ordinals.
+template <typename Kern>
+static cudaError_t smem_opt_in(Kern kern, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 template <int DT, int IMG, int BN, int OUT, int XKB>
 static cudaError_t launch_t(const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
                             const Plan& p, const SpmmArgs& a, cudaStream_t s) {
   using C = Cfg<DT, IMG, BN, OUT, XKB>;
   auto kern = spmm_kernel<DT, IMG, BN, OUT, XKB>;
-  static bool attr_set = false;  // per instantiation; set once per process (single device use)
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> opted{0};
+  cudaError_t e = smem_opt_in(kern, C::SMEM, opted);
+  if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(p.grid), C::THREADS, C::SMEM, s, *tmX, *tmY, *tmW, a);
 }
 
@@ -1067,12 +1079,9 @@ static cudaError_t launch_pair_t(const CUtensorMap* tmX, const CUtensorMap* tmY,
                                  const Plan& p, const SpmmArgs& a, cudaStream_t s) {
   using C = PairCfg<DT, IMG, BN, OUT>;
   auto kern = spmm_pair_kernel<DT, IMG, BN, OUT>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> opted{0};
+  cudaError_t e = smem_opt_in(kern, C::SMEM, opted);
+  if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(2 * p.grid), C::THREADS, C::SMEM, s, *tmX, *tmY, *tmW, a);  // p.grid = CTA pairs
 }
 
@@ -1141,14 +1150,18 @@ cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const CUtens
   return a.tma_store ? launch_dt<0>(h, tmX, tmY, tmW, p, a, s) : launch_dt<kOutDirect>(h, tmX, tmY, tmW, p, a, s);
 }
 
-// Pairs that can be resident at once for a pair-kernel configuration (cached).
+// Pairs that can be resident at once for a pair-kernel configuration (cached per device).
 template <int DT, int IMG, int BN, int OUT>
 static int max_clusters_t() {
-  static int cached = 0;
+  static std::atomic<int> cache[64];
+  static std::atomic<uint64_t> opted{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  int cached = cache[dev].load(std::memory_order_acquire);
   if (!cached) {
     using C = PairCfg<DT, IMG, BN, OUT>;
     auto kern = spmm_pair_kernel<DT, IMG, BN, OUT>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (smem_opt_in(kern, C::SMEM, opted) != cudaSuccess) cudaGetLastError();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(C::THREADS, 1, 1);
@@ -1161,6 +1174,7 @@ static int max_clusters_t() {
       n = 0;
     }
     cached = n > 0 ? n : -1;
+    cache[dev].store(cached, std::memory_order_release);
   }
   return cached;
 }
