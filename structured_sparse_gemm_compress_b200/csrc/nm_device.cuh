@@ -120,6 +120,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// True in exactly one lane of a converged warp (the lowest active lane).  The
+// tcgen05 operations that one thread must issue are issued by that lane while
+// the loop around them, and the descriptors they take, stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// mbar_wait by every lane of a warp; the warp gives up (false in all lanes) if
+// any lane gave up, so the decision stays warp-uniform.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                               uint64_t timeout_ns) {
+  const bool got = mbar_wait(bar, parity, abort, timeout_ns);
+  return __all_sync(0xffffffffu, got) != 0;
+}
+
 // One contiguous global -> shared copy completing on `bar` (16-byte aligned, size % 16 == 0).
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile(

@@ -21,7 +21,7 @@
 // CTA = 2 + 4 * epw warps, one persistent CTA per SM:
 //   warp 0      producer: one bulk copy of the packed weight chunk (values +
 //               positions) and two 2-D tensor copies of X per stage;
-//   warp 1      TMEM owner and MMA issuer (one thread): copies the positions
+//   warp 1      TMEM owner and MMA issuer (one elected lane): copies the positions
 //               into TMEM (tcgen05.cp) and issues tcgen05.mma(.sp);
 //   warps 2..   epilogue, epw warps per TMEM lane quarter (each owning BN/epw
 //               token columns): tcgen05.ld, the output stage, then coalesced
@@ -468,7 +468,10 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (barrier waits, descriptors); one elected
+    // lane issues the tcgen05 copies, MMAs and commits.
+    {
+      const bool issuer = elect_one();
       constexpr uint32_t idesc = make_idesc<DT, SP, BN>();
       int stage = 0, acc = 0, eslot = 0, cur_tt = -1, mseq = 0, mtile = 0;
       uint32_t phase = 0, acc_phase = 0, xphase = 0;
@@ -476,29 +479,29 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
       for (int u = ur.first; ok && u < ur.end; u += ur.step) {
         const Unit w = decode_unit(u, a);
         if (XS && w.tt != cur_tt) {
-          if (cur_tt >= 0) tc_commit(&xempty_bar);  // the old X tile is free once these MMAs finish
-          if (!mbar_wait(&xfull_bar, xphase, &abort_sh, tmo)) {
-            give_up(3);
+          if (cur_tt >= 0 && issuer) tc_commit(&xempty_bar);  // the old X tile is free once these MMAs finish
+          if (!mbar_wait_warp(&xfull_bar, xphase, &abort_sh, tmo)) {
+            if (issuer) give_up(3);
             break;
           }
           xphase ^= 1u;
           cur_tt = w.tt;
         }
-        if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &abort_sh, tmo)) {
-          give_up(2);
+        if (!mbar_wait_warp(&acce_bar[acc], acc_phase ^ 1u, &abort_sh, tmo)) {
+          if (issuer) give_up(2);
           break;
         }
-        NM_TR(TR_M_ACCE, mtile);
+        if (issuer) NM_TR(TR_M_ACCE, mtile);
         ++mtile;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_sh, tmo)) {
-            give_up(3);
+          if (!mbar_wait_warp(&full_bar[stage], phase, &abort_sh, tmo)) {
+            if (issuer) give_up(3);
             ok = false;
             break;
           }
-          NM_TR(TR_M_FULL, mseq);
+          if (issuer) NM_TR(TR_M_FULL, mseq);
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + (size_t)stage * C::STAGE);
           const uint32_t b_addr = XS ? smem_u32(xregion + (size_t)kb * C::B_KBLK) : a_addr + C::CHUNK;
@@ -506,10 +509,12 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
           if constexpr (SP) {
             e_tmem = tmem + (uint32_t)(C::E_COL0 + eslot * C::E_COLS);
             const uint32_t e_addr = a_addr + kAtomBytes;
-            if constexpr (DT == DT_I8)
-              tc_cp_128x256b(e_tmem, sdesc_rows16x2(e_addr));
-            else
-              tc_cp_128x128b(e_tmem, sdesc_rows16(e_addr));
+            if (issuer) {
+              if constexpr (DT == DT_I8)
+                tc_cp_128x256b(e_tmem, sdesc_rows16x2(e_addr));
+              else
+                tc_cp_128x128b(e_tmem, sdesc_rows16(e_addr));
+            }
           }
           // descriptors differ only in the start-address field: build once, add offsets
           const uint64_t ad0 = sdesc_sw128(a_addr), bd0 = sdesc_sw128(b_addr);
@@ -527,15 +532,15 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
                 e_addr = e_tmem + (uint32_t)(j & ~1);
                 id2 = (uint32_t)(j & 1);
               }
-              tc_mma_sp<KIND>(d_tmem, ad, bd, e_addr, idesc | id2, accum);
+              if (issuer) tc_mma_sp<KIND>(d_tmem, ad, bd, e_addr, idesc | id2, accum);
             } else {
               const uint64_t ad = ad0 + (uint64_t)(((uint32_t)((j >> 2) * kAtomBytes) + 32u * (j & 3)) >> 4);
               const uint64_t bd = bd0 + (uint64_t)(((uint32_t)((j >> 2) * C::B_BOX) + 32u * (j & 3)) >> 4);
-              tc_mma<KIND>(d_tmem, ad, bd, idesc, accum);
+              if (issuer) tc_mma<KIND>(d_tmem, ad, bd, idesc, accum);
             }
           }
-          tc_commit(&empty_bar[stage]);  // frees the smem stage once these MMAs have read it
-          NM_TR(TR_M_DONE, mseq);
+          if (issuer) tc_commit(&empty_bar[stage]);  // frees the smem stage once these MMAs have read it
+          if (issuer) NM_TR(TR_M_DONE, mseq);
           ++mseq;
           eslot ^= 1;
           if (++stage == C::STAGES) {
@@ -544,15 +549,15 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
           }
         }
         if (!ok) break;
-        tc_commit(&accf_bar[acc]);  // accumulator ready for the epilogue
+        if (issuer) tc_commit(&accf_bar[acc]);  // accumulator ready for the epilogue
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
-      // Drain: all tcgen05 work issued by this thread completes before TMEM is freed.
-      tc_commit(&drain_bar);
-      mbar_wait(&drain_bar, 0, &abort_sh, tmo);
+      // Drain: all tcgen05 work issued by this warp completes before TMEM is freed.
+      if (issuer) tc_commit(&drain_bar);
+      mbar_wait_warp(&drain_bar, 0, &abort_sh, tmo);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -856,25 +861,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
-    if (lane == 0 && leader) {
+    // The leader's whole warp runs the loop; one elected lane issues.
+    if (leader) {
+      const bool issuer = elect_one();
       constexpr uint32_t idesc = make_idesc<DT, SP, BN, 256>();
       int stage = 0, acc = 0, eslot = 0, mseq = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int u = u_first; ok && u < a.units; u += u_step) {
-        if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &abort_sh, tmo)) {
-          give_up(2);
+        if (!mbar_wait_warp(&acce_bar[acc], acc_phase ^ 1u, &abort_sh, tmo)) {
+          if (issuer) give_up(2);
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < a.n_kb; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_sh, tmo)) {
-            give_up(3);
+          if (!mbar_wait_warp(&full_bar[stage], phase, &abort_sh, tmo)) {
+            if (issuer) give_up(3);
             ok = false;
             break;
           }
-          NM_TR(TR_M_FULL, mseq);
+          if (issuer) NM_TR(TR_M_FULL, mseq);
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + (size_t)stage * C::STAGE);
           const uint32_t b_addr = a_addr + C::CHUNK;
@@ -882,10 +889,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
           if constexpr (SP) {
             e_tmem = tmem + (uint32_t)(C::E_COL0 + eslot * C::E_COLS);
             const uint32_t e_addr = a_addr + kAtomBytes;
-            if constexpr (DT == DT_I8)
-              tc_cp_128x256b_pair(e_tmem, sdesc_rows16x2(e_addr));
-            else
-              tc_cp_128x128b_pair(e_tmem, sdesc_rows16(e_addr));
+            if (issuer) {
+              if constexpr (DT == DT_I8)
+                tc_cp_128x256b_pair(e_tmem, sdesc_rows16x2(e_addr));
+              else
+                tc_cp_128x128b_pair(e_tmem, sdesc_rows16(e_addr));
+            }
           }
           const uint64_t ad0 = sdesc_sw128(a_addr), bd0 = sdesc_sw128(b_addr);
 #pragma unroll
@@ -902,15 +911,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
                 e_addr = e_tmem + (uint32_t)(j & ~1);
                 id2 = (uint32_t)(j & 1);
               }
-              tc_mma_sp_pair<KIND>(d_tmem, ad, bd, e_addr, idesc | id2, accum);
+              if (issuer) tc_mma_sp_pair<KIND>(d_tmem, ad, bd, e_addr, idesc | id2, accum);
             } else {
               const uint64_t ad = ad0 + (uint64_t)(((uint32_t)((j >> 2) * kAtomBytes) + 32u * (j & 3)) >> 4);
               const uint64_t bd = bd0 + (uint64_t)(((uint32_t)((j >> 2) * C::B_BOX) + 32u * (j & 3)) >> 4);
-              tc_mma_pair<KIND>(d_tmem, ad, bd, idesc, accum);
+              if (issuer) tc_mma_pair<KIND>(d_tmem, ad, bd, idesc, accum);
             }
           }
-          tc_commit_pair(&empty_bar[stage], (uint16_t)3);  // frees this stage in both CTAs
-          NM_TR(TR_M_DONE, mseq);
+          if (issuer) tc_commit_pair(&empty_bar[stage], (uint16_t)3);  // frees this stage in both CTAs
+          if (issuer) NM_TR(TR_M_DONE, mseq);
           ++mseq;
           eslot ^= 1;
           if (++stage == C::STAGES) {
@@ -919,16 +928,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
           }
         }
         if (!ok) break;
-        tc_commit_pair(&accf_bar[acc], (uint16_t)3);  // both CTAs' accumulators are ready
+        if (issuer) tc_commit_pair(&accf_bar[acc], (uint16_t)3);  // both CTAs' accumulators are ready
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
-      tc_commit_pair(&drain_bar, (uint16_t)3);  // every MMA of this pair has completed
-      mbar_wait(&drain_bar, 0, &abort_sh, tmo);
-    } else if (lane == 0) {
-      mbar_wait(&drain_bar, 0, &abort_sh, tmo);  // peer: the leader's MMAs into this TMEM are done
+      if (issuer) tc_commit_pair(&drain_bar, (uint16_t)3);  // every MMA of this pair has completed
+      mbar_wait_warp(&drain_bar, 0, &abort_sh, tmo);
+    } else {
+      mbar_wait_warp(&drain_bar, 0, &abort_sh, tmo);  // peer: the leader's MMAs into this TMEM are done
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
