@@ -405,7 +405,9 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues the copies.
+    {
+      const bool issuer = elect_one();
       int stage = 0, seq = 0, cur_tt = -1;
       uint32_t phase = 0, xphase = 0;
       uint32_t armed = 0, armed_par = 0;  // per stage: last use carried copies / its parity
@@ -415,38 +417,43 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
         const Unit w = decode_unit(u, a);
         if (XS && w.tt != cur_tt) {
           // load the X tile of this token tile once the MMAs on the previous one have completed
-          if (!mbar_wait(&xempty_bar, xphase ^ 1u, &abort_sh, tmo)) {
-            give_up(1);
+          if (!mbar_wait_warp(&xempty_bar, xphase ^ 1u, &abort_sh, tmo)) {
+            if (issuer) give_up(1);
             break;
           }
-          mbar_arrive_expect_tx(&xfull_bar, (uint32_t)(a.n_kb * C::B_KBLK));
-          for (int kb = 0; kb < a.n_kb; ++kb) {
-            uint8_t* xs = xregion + (size_t)kb * C::B_KBLK;
-            tma_load_2d(xs, &tmX, &xfull_bar, kb * C::KB, w.tt * BN);
-            tma_load_2d(xs + C::B_BOX, &tmX, &xfull_bar, kb * C::KB + C::KB / 2, w.tt * BN);
+          if (issuer) {
+            mbar_arrive_expect_tx(&xfull_bar, (uint32_t)(a.n_kb * C::B_KBLK));
+            for (int kb = 0; kb < a.n_kb; ++kb) {
+              uint8_t* xs = xregion + (size_t)kb * C::B_KBLK;
+              tma_load_2d(xs, &tmX, &xfull_bar, kb * C::KB, w.tt * BN);
+              tma_load_2d(xs + C::B_BOX, &tmX, &xfull_bar, kb * C::KB + C::KB / 2, w.tt * BN);
+            }
           }
           xarmed = true;
           xphase ^= 1u;
           cur_tt = w.tt;
         }
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++seq) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
-            give_up(1);
+          if (!mbar_wait_warp(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
+            if (issuer) give_up(1);
             ok = false;
             break;
           }
-          NM_TR(TR_P_ISSUE, seq);
+          if (issuer) NM_TR(TR_P_ISSUE, seq);
           if (seq != a.inject_skip) {
             uint8_t* st = smem + (size_t)stage * C::STAGE;
-            mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)C::STAGE);
-            if (a.w_tma)  // the packed image as rows of 128 bytes: one box = one chunk
-              tma_load_2d(st, &tmW, &full_bar[stage], 0, (w.ct * a.n_kb + kb) * (C::CHUNK / 128));
-            else
-              bulk_load(st, a.bpack + ((size_t)w.ct * a.n_kb + kb) * C::CHUNK, (uint32_t)C::CHUNK,
-                        &full_bar[stage]);
-            if constexpr (!XS) {
-              tma_load_2d(st + C::CHUNK, &tmX, &full_bar[stage], kb * C::KB, w.tt * BN);
-              tma_load_2d(st + C::CHUNK + C::B_BOX, &tmX, &full_bar[stage], kb * C::KB + C::KB / 2, w.tt * BN);
+            const int wrow = (w.ct * a.n_kb + kb) * (C::CHUNK / 128);
+            if (issuer) {
+              mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)C::STAGE);
+              if (a.w_tma)  // the packed image as rows of 128 bytes: one box = one chunk
+                tma_load_2d(st, &tmW, &full_bar[stage], 0, wrow);
+              else
+                bulk_load(st, a.bpack + ((size_t)w.ct * a.n_kb + kb) * C::CHUNK, (uint32_t)C::CHUNK,
+                          &full_bar[stage]);
+              if constexpr (!XS) {
+                tma_load_2d(st + C::CHUNK, &tmX, &full_bar[stage], kb * C::KB, w.tt * BN);
+                tma_load_2d(st + C::CHUNK + C::B_BOX, &tmX, &full_bar[stage], kb * C::KB + C::KB / 2, w.tt * BN);
+              }
             }
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -459,12 +466,12 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
           }
         }
       }
-      // Drain: every copy this thread issued has landed before the CTA exits.
+      // Drain: every copy this warp issued has landed before the CTA exits.
       // Earlier uses of a stage were consumed before it was re-armed, so only
       // the last armed use of each stage (and the last X tile) can still be in flight.
       for (int i = 0; i < C::STAGES; ++i)
-        if ((armed >> i) & 1u) mbar_wait(&full_bar[i], (armed_par >> i) & 1u, &abort_sh, tmo);
-      if (xarmed) mbar_wait(&xfull_bar, xphase ^ 1u, &abort_sh, tmo);
+        if ((armed >> i) & 1u) mbar_wait_warp(&full_bar[i], (armed_par >> i) & 1u, &abort_sh, tmo);
+      if (xarmed) mbar_wait_warp(&xfull_bar, xphase ^ 1u, &abort_sh, tmo);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -819,7 +826,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues the copies.
+    {
+      const bool issuer = elect_one();
       int stage = 0, seq = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
@@ -828,20 +837,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
         const int pt = u % n_pct, tt = u / n_pct;
         const int ct = 2 * pt + (int)rank;
         for (int kb = 0; kb < a.n_kb; ++kb, ++seq) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
-            give_up(1);
+          if (!mbar_wait_warp(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
+            if (issuer) give_up(1);
             ok = false;
             break;
           }
-          NM_TR(TR_P_ISSUE, seq);
+          if (issuer) NM_TR(TR_P_ISSUE, seq);
           if (seq != a.inject_skip) {
             uint8_t* st = smem + (size_t)stage * C::STAGE;
             const uint32_t fb = full_lead0 + 8u * (uint32_t)stage;
-            if (leader) mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)(2 * C::STAGE));
-            tma_load_2d_pair(st, &tmW, fb, 0, (ct * a.n_kb + kb) * (C::CHUNK / 128));
-            tma_load_2d_pair(st + C::CHUNK, &tmX, fb, kb * C::KB, tt * BN + (int)rank * C::HB);
-            tma_load_2d_pair(st + C::CHUNK + C::B_BOX, &tmX, fb, kb * C::KB + C::KB / 2,
-                             tt * BN + (int)rank * C::HB);
+            const int wrow = (ct * a.n_kb + kb) * (C::CHUNK / 128);
+            const int trow = tt * BN + (int)rank * C::HB;
+            if (issuer) {
+              if (leader) mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)(2 * C::STAGE));
+              tma_load_2d_pair(st, &tmW, fb, 0, wrow);
+              tma_load_2d_pair(st + C::CHUNK, &tmX, fb, kb * C::KB, trow);
+              tma_load_2d_pair(st + C::CHUNK + C::B_BOX, &tmX, fb, kb * C::KB + C::KB / 2, trow);
+            }
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           } else {
@@ -857,7 +869,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
       // held by the cluster barrier below until the leader has seen them land.
       if (leader)
         for (int i = 0; i < C::STAGES; ++i)
-          if ((armed >> i) & 1u) mbar_wait(&full_bar[i], (armed_par >> i) & 1u, &abort_sh, tmo);
+          if ((armed >> i) & 1u) mbar_wait_warp(&full_bar[i], (armed_par >> i) & 1u, &abort_sh, tmo);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
