@@ -577,21 +577,35 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
         smem + (size_t)C::STAGES * C::STAGE + C::X_BYTES + (size_t)ew * C::EPI_NB * C::EPI_BUF;
     int buf = 0, acc = 0;
     uint32_t acc_phase = 0;
-    // One thread waits (bounded) and broadcasts the outcome, so all epilogue
-    // threads take the same branch and always meet at the named barriers; the
-    // flag alternates between two slots so a fast thread's next write cannot
-    // overtake a slow thread's read.
+    // Runtime-stage kernels without split-K: each warp waits (bounded, warp
+    // vote) for its tile's accumulator on its own.  Otherwise one thread waits
+    // and broadcasts the outcome and every thread takes the same branch (the
+    // split-K path meets at named barriers); the flag alternates between two
+    // slots so a fast thread's next write cannot overtake a slow thread's read.
     int iter = 0;
     for (int u = ur.first; u < ur.end; u += ur.step, ++iter) {
       const Unit w = decode_unit(u, a);
-      if (ep_tid == 0) {
-        const bool got = mbar_wait(&accf_bar[acc], acc_phase, &abort_sh, tmo);
-        if (!got) give_up(4);
-        ep_ok_sh[iter & 1] = got ? 1 : 0;
-        NM_TR(TR_E_START, iter);
+      if (EPI && a.splits == 1) {
+        // No named barrier below: each warp waits for the accumulator itself
+        // (measured faster for the runtime output stage, slower for the fixed
+        // fp32 stage, whose warps stay in step through the shared wait).
+        if (!mbar_wait_warp(&accf_bar[acc], acc_phase, &abort_sh, tmo)) {
+          if (lane == 0) give_up(4);
+          break;
+        }
+        if (ep_tid == 0) NM_TR(TR_E_START, iter);
+      } else {
+        // The split-K path meets at named barriers: every warp must take the
+        // same branch, so one thread decides and broadcasts.
+        if (ep_tid == 0) {
+          const bool got = mbar_wait(&accf_bar[acc], acc_phase, &abort_sh, tmo);
+          if (!got) give_up(4);
+          ep_ok_sh[iter & 1] = got ? 1 : 0;
+          NM_TR(TR_E_START, iter);
+        }
+        named_bar_sync(1, 32 * C::EPI_WARPS);
+        if (!ep_ok_sh[iter & 1]) break;
       }
-      named_bar_sync(1, 32 * C::EPI_WARPS);
-      if (!ep_ok_sh[iter & 1]) break;
       tc_fence_after();
       const int ch0 = w.ct * kRows + lq * 32;  // first channel of this warp's lane quarter
       const int ch = ch0 + lane;
@@ -778,7 +792,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
-  __shared__ volatile int ep_ok_sh[2];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -964,14 +977,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
     for (int u = u_first; u < a.units; u += u_step, ++iter) {
       const int pt = u % n_pct, tt = u / n_pct;
       const int ct = 2 * pt + (int)rank;
-      if (ep_tid == 0) {
-        const bool got = mbar_wait(&accf_bar[acc], acc_phase, &abort_sh, tmo);
-        if (!got) give_up(4);
-        ep_ok_sh[iter & 1] = got ? 1 : 0;
-        NM_TR(TR_E_START, iter);
+      // No named barrier in this loop: each warp waits for the accumulator itself.
+      if (!mbar_wait_warp(&accf_bar[acc], acc_phase, &abort_sh, tmo)) {
+        if (lane == 0) give_up(4);
+        break;
       }
-      named_bar_sync(1, 32 * C::EPI_WARPS);
-      if (!ep_ok_sh[iter & 1]) break;
+      if (ep_tid == 0) NM_TR(TR_E_START, iter);
       tc_fence_after();
       const int ch0 = ct * kRows + lq * 32;
       const int ch = ch0 + lane;
