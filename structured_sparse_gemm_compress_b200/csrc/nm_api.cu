@@ -365,7 +365,8 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   int oes, oty;
   out_type(h, scale != nullptr, &oes, &oty);
   const int wcols = p.bn / nm::epw_for(false);  // token columns per epilogue warp; the TMA-store box
-  const int ych = p.pair ? (wcols % 32 == 0 ? 32 : wcols % 16 == 0 ? 16 : 8) : std::min(32, wcols);
+  const int ych = p.pair ? (wcols % 32 == 0 ? 32 : wcols % 16 == 0 ? 16 : 8)
+                         : (wcols % 32 == 0 ? 32 : (wcols % 8 == 0 && wcols <= 96) ? wcols : 8);
   // Direct stores measured faster than staged TMA stores (they keep the TMA unit
   // for operand loads); the TMA-store epilogue remains selectable.
   a.tma_store = 0;
@@ -647,7 +648,8 @@ nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y
   int oes, oty;
   out_type(h, scale != nullptr, &oes, &oty);
   const int wcols = p.bn / nm::epw_for(false);  // token columns per epilogue warp; the TMA-store box
-  const int ych = p.pair ? (wcols % 32 == 0 ? 32 : wcols % 16 == 0 ? 16 : 8) : std::min(32, wcols);
+  const int ych = p.pair ? (wcols % 32 == 0 ? 32 : wcols % 16 == 0 ? 16 : 8)
+                         : (wcols % 32 == 0 ? 32 : (wcols % 8 == 0 && wcols <= 96) ? wcols : 8);
   // Direct stores measured faster than staged TMA stores (they keep the TMA unit
   // for operand loads); the TMA-store epilogue remains selectable.
   a.tma_store = 0;

@@ -81,7 +81,8 @@ struct Cfg {
   static constexpr int EPI_WARPS = epi_warps(OUT);
   static constexpr int THREADS = cta_threads(OUT);
   static constexpr int WCOLS = BN / (EPI_WARPS / 4);
-  static constexpr int CH = (WCOLS % 32 == 0) ? 32 : (WCOLS % 16 == 0) ? 16 : 8;
+  // chunks of 32 columns, or one chunk of the whole run when it is not a multiple of 32
+  static constexpr int CH = (WCOLS % 32 == 0) ? 32 : (WCOLS % 8 == 0 && WCOLS <= 96) ? WCOLS : 8;
   static constexpr int NCH = WCOLS / CH;
   static constexpr int OES = out_bytes(OUT);
   static constexpr int EPI_BUF = CH * 32 * OES;     // one staged [CH tokens][32 channels] tile
@@ -323,15 +324,27 @@ __device__ __forceinline__ uint32_t add_acc(uint32_t x, uint32_t y) {
     return __float_as_uint(__uint_as_float(x) + __uint_as_float(y));
 }
 
+// N consecutive 32-bit columns of this warp's 32 lanes, N a multiple of 8:
+// issued as 32-, 16- and 8-column loads with no wait in between (the caller
+// waits once with tmem_wait_ld).
+template <int N, int OFF = 0>
+__device__ __forceinline__ void tmem_ld_run(uint32_t taddr, uint32_t* r) {
+  if constexpr (N - OFF >= 32) {
+    tmem_ld32(taddr + OFF, *reinterpret_cast<uint32_t(*)[32]>(r + OFF));
+    tmem_ld_run<N, OFF + 32>(taddr, r);
+  } else if constexpr (N - OFF >= 16) {
+    tmem_ld16(taddr + OFF, *reinterpret_cast<uint32_t(*)[16]>(r + OFF));
+    tmem_ld_run<N, OFF + 16>(taddr, r);
+  } else if constexpr (N - OFF >= 8) {
+    tmem_ld8(taddr + OFF, *reinterpret_cast<uint32_t(*)[8]>(r + OFF));
+    tmem_ld_run<N, OFF + 8>(taddr, r);
+  }
+}
+
 template <int N>
 __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]) {
-  static_assert(N == 8 || N == 16 || N == 32, "tcgen05.ld width");
-  if constexpr (N == 32)
-    tmem_ld32(taddr, r);
-  else if constexpr (N == 16)
-    tmem_ld16(taddr, r);
-  else
-    tmem_ld8(taddr, r);
+  static_assert(N % 8 == 0 && N <= 96, "tcgen05.ld run width");
+  tmem_ld_run<N>(taddr, r);
 }
 
 template <int DT, int IMG, int BN, int OUT, int XKB>
