@@ -101,6 +101,154 @@ __device__ __forceinline__ void store_bytes(uint8_t* dst, const uint32_t* w, int
   }
 }
 
+// INT8 fast path for a full unit of 16 positions held as four 32-bit words
+// (byte i of word j is position 4j + i).  The kept set comes from a rank per
+// position -- how many positions of its group precede it in the order
+// (|w| descending, position ascending), kept iff fewer than N -- computed by
+// pairwise compares; kept values are gathered with byte permutes.
+template <int N, int M>
+__device__ __forceinline__ uint32_t keep_mask_i8(const uint32_t (&w)[4]) {
+  if constexpr (N == M) {
+    return 0xFFFFu;
+  } else {
+    uint32_t mag[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int v = (int)(int8_t)(uint8_t)(w[c >> 2] >> (8 * (c & 3)));
+      mag[c] = (uint32_t)(v < 0 ? -v : v);
+    }
+    uint32_t keep = 0;
+#pragma unroll
+    for (int g = 0; g < 16 / M; ++g) {
+      int rank[M];
+#pragma unroll
+      for (int i = 0; i < M; ++i) rank[i] = 0;
+#pragma unroll
+      for (int p = 0; p < M; ++p)
+#pragma unroll
+        for (int q = p + 1; q < M; ++q) {
+          // q (the later position) precedes p only with a strictly larger magnitude
+          const int later_first = mag[g * M + q] > mag[g * M + p] ? 1 : 0;
+          rank[p] += later_first;
+          rank[q] += 1 - later_first;
+        }
+#pragma unroll
+      for (int p = 0; p < M; ++p) keep |= (rank[p] < N ? 1u : 0u) << (g * M + p);
+    }
+    return keep;
+  }
+}
+
+// Bytes of the kept positions of bits `m` (group-relative, ascending) as a
+// byte-permute selector over the group's words; also their 4-bit positions.
+template <int N>
+__device__ __forceinline__ void kept_selector(uint32_t m, uint32_t& sel, uint32_t& nib) {
+  sel = 0x4444u;  // nibble 4..7 select bytes of the zero second operand
+  nib = 0;
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const uint32_t p = (uint32_t)(__ffs(m) - 1);
+    m &= m - 1u;
+    sel = (sel & ~(0xFu << (4 * j))) | (p << (4 * j));
+    nib |= p << (4 * j);
+  }
+}
+
+template <int N, int M, int IMG>
+__device__ __forceinline__ void compress_unit_i8(const uint32_t (&w)[4], int64_t r, int64_t k0, int64_t K,
+                                                 int n_kb, int8_t* __restrict__ values, uint8_t* __restrict__ idx,
+                                                 int64_t idx_pitch, uint8_t* __restrict__ bpack) {
+  constexpr int G = 16 / M;
+  constexpr int CNT = 16 * N / M;
+  const uint32_t keep = keep_mask_i8<N, M>(w);
+
+  // ---- canonical format
+  uint32_t vw[(CNT + 3) / 4] = {};
+  uint32_t nibw[(CNT + 7) / 8 > 0 ? (CNT + 7) / 8 : 1] = {};
+  if constexpr (N == M) {  // everything kept: the values are the unit itself
+#pragma unroll
+    for (int i = 0; i < 4; ++i) vw[i] = w[i];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) nibw[e / 8] |= (uint32_t)(e % M) << (4 * (e % 8));
+  } else {
+    static_assert(N <= 4, "one byte permute gathers at most four kept values");
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      uint32_t sel, nib;
+      kept_selector<N>((keep >> (g * M)) & ((1u << M) - 1u), sel, nib);
+      uint32_t v;
+      if constexpr (M == 4)
+        v = __byte_perm(w[g], 0u, sel);
+      else
+        v = __byte_perm(w[2 * g], w[2 * g + 1], sel & 0x7777u);  // positions 0..7 of the pair
+      const int e0 = g * N;  // first kept element of this group within the unit
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const int e = e0 + j;
+        vw[e / 4] |= ((v >> (8 * j)) & 0xFFu) << (8 * (e % 4));
+        nibw[e / 8] |= ((nib >> (4 * j)) & 0xFu) << (4 * (e % 8));
+      }
+    }
+  }
+  const int64_t kept_per_row = (K / M) * N;
+  const int64_t e0 = (k0 / M) * N;
+  uint8_t* vdst = reinterpret_cast<uint8_t*>(values + r * kept_per_row + e0);
+  uint8_t* idst = idx + r * idx_pitch + e0 / 2;
+  if constexpr (CNT >= 4) {
+    store_bytes(vdst, vw, CNT);
+  } else {
+    for (int b = 0; b < CNT; ++b) vdst[b] = (uint8_t)(vw[0] >> (8 * b));
+  }
+  if constexpr (CNT / 2 >= 4) {
+    store_bytes(idst, nibw, CNT / 2);
+  } else {
+    for (int b = 0; b < CNT / 2; ++b) idst[b] = (uint8_t)(nibw[0] >> (8 * b));
+  }
+
+  // ---- packed operand image
+  const int64_t ct = r / kRows;
+  const uint32_t rr = (uint32_t)(r % kRows);
+  const int kb = (int)(k0 / kblock_elems(DT_I8));
+  const uint32_t kk = (uint32_t)(k0 % kblock_elems(DT_I8));
+  uint8_t* chunk = bpack + ((size_t)ct * n_kb + kb) * (size_t)chunk_bytes(DT_I8, IMG);
+  if constexpr (IMG == IMG_SP24) {
+    uint32_t comp[2] = {0u, 0u}, meta = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // groups of four: two slots each, positions ascending
+      const uint32_t bits = (keep >> (4 * j)) & 0xFu;
+      const int n = __popc(bits);
+      const uint32_t lo = (uint32_t)(__ffs(bits) - 1);
+      const uint32_t hi = (uint32_t)(31 - __clz(bits | 1u));
+      uint32_t i0, i1, sel;  // slot positions; selector (4 = a zero byte)
+      if (n >= 2) {
+        i0 = lo; i1 = hi; sel = lo | (hi << 4);
+      } else if (n == 1 && lo < 3) {
+        i0 = lo; i1 = 3; sel = lo | (4u << 4);
+      } else if (n == 1) {
+        i0 = 0; i1 = 3; sel = 4u | (3u << 4);
+      } else {
+        i0 = 0; i1 = 1; sel = 4u | (4u << 4);
+      }
+      const uint32_t two = __byte_perm(w[j], 0u, sel | 0x4400u) & 0xFFFFu;
+      comp[j >> 1] |= two << (16 * (j & 1));
+      meta |= (i0 | (i1 << 2)) << (4 * j);
+    }
+    *reinterpret_cast<uint2*>(chunk + swz128(rr, kk / 2)) = make_uint2(comp[0], comp[1]);
+    *reinterpret_cast<uint16_t*>(chunk + kAtomBytes + meta_off16(DT_I8, rr, kk)) = (uint16_t)meta;
+  } else {
+    uint32_t d[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t b4 = (keep >> (4 * j)) & 0xFu;  // one bit per byte of word j
+      const uint32_t bytemask = ((b4 & 1u) ? 0xFFu : 0u) | ((b4 & 2u) ? 0xFF00u : 0u) |
+                                ((b4 & 4u) ? 0xFF0000u : 0u) | ((b4 & 8u) ? 0xFF000000u : 0u);
+      d[j] = w[j] & bytemask;
+    }
+    *reinterpret_cast<uint4*>(chunk + (kk >> 7) * kAtomBytes + swz128(rr, kk & 127u)) =
+        make_uint4(d[0], d[1], d[2], d[3]);
+  }
+}
+
 template <int DT, int N, int M>
 __global__ void __launch_bounds__(256) compress_kernel(const typename Elem<DT>::T* __restrict__ W, int64_t n_out,
                                                        int64_t K, int n_kb, typename Elem<DT>::T* __restrict__ values,
@@ -123,6 +271,14 @@ __global__ void __launch_bounds__(256) compress_kernel(const typename Elem<DT>::
   const int64_t rem = K - k0;
   const int valid = r < n_out ? (int)(rem < 0 ? 0 : (rem > 16 ? 16 : rem)) : 0;
   const T* src = W + r * K + k0;
+  if constexpr (DT == DT_I8) {
+    if (valid == 16 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(src));
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      compress_unit_i8<N, M, IMG>(w, r, k0, K, n_kb, reinterpret_cast<int8_t*>(values), idx, idx_pitch, bpack);
+      return;
+    }
+  }
   if (valid == 16 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
 #pragma unroll
     for (int h = 0; h < ES; ++h) unpack16<T>(__ldg(reinterpret_cast<const uint4*>(src) + h), raw + h * (16 / ES));
