@@ -20,7 +20,11 @@ arrays, and states the readings of the paper that the C code follows:
 * top-N by magnitude, ties to the lower in-group position;
 * exactly N slots per group, kept values in ascending position;
 * ``idx`` holds one 4-bit position per kept element, two per byte, low nibble
-  first, each row padded to whole bytes.
+  first, each row padded to whole bytes;
+* tile-shared compress (``compress_tile``, the vector-wise reading of the
+  micro-dense format): the rows of a tile of consecutive output channels keep
+  one pattern, chosen by the same rule with the tile's column mass (sum of |w|)
+  as the magnitude, so that one gather of the activations serves the tile.
 """
 from __future__ import annotations
 
@@ -55,6 +59,7 @@ def _load():
         lib = ctypes.CDLL(build())
         i64, p, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
         lib.oracle_compress.argtypes = [p, i64, i64, i32, i32, i32, p, p]
+        lib.oracle_compress_tile.argtypes = [p, i64, i64, i32, i32, i32, i64, p, p]
         lib.oracle_decompress.argtypes = [p, p, i64, i64, i32, i32, i32, p]
         lib.oracle_gemm_i8.argtypes = [p, i64, i64, p, i64, p, p, p]
         lib.oracle_gemm_f16.argtypes = [p, i64, i64, p, i64, i32, p, p]
@@ -112,6 +117,23 @@ def compress(W: np.ndarray, N: int, M: int, dtype: str | None = None):
     rc = _load().oracle_compress(_ptr(W), n_out, k, code, N, M, _ptr(values), _ptr(idx))
     if rc != 0:
         raise ValueError(f"oracle_compress rejected the arguments (rc={rc})")
+    return values, idx
+
+
+def compress_tile(W: np.ndarray, N: int, M: int, tile: int = 128, dtype: str | None = None):
+    """Tile-shared top-N-of-M compression: the rows of each tile of ``tile``
+    consecutive rows keep the same positions, those of largest column mass
+    (sum of |w| over the tile), ties to the lower position.  int8 or float16
+    only.  Same return layout as ``compress``.
+    """
+    W = np.ascontiguousarray(W)
+    n_out, k = W.shape
+    code = _dtype_code(W, dtype)
+    values = np.zeros((n_out, k // M, N), dtype=W.dtype)
+    idx = np.zeros((n_out, idx_pitch(k, N, M)), dtype=np.uint8)
+    rc = _load().oracle_compress_tile(_ptr(W), n_out, k, code, N, M, tile, _ptr(values), _ptr(idx))
+    if rc != 0:
+        raise ValueError(f"oracle_compress_tile rejected the arguments (rc={rc})")
     return values, idx
 
 

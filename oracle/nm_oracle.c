@@ -28,11 +28,18 @@
  *     requantisation): the library's own definition, see oracle_epilogue_i8;
  *     the paper does not discuss the output stage.
  *
+ * Tile-shared compress (oracle_compress_tile): the same top-N rule with the
+ * column mass of a tile of V rows as the magnitude, so a tile's rows share one
+ * pattern (the vector-wise reading; the paper does not fix the granularity).
+ *
  * Parity pins (tests/test_oracle.py): hand-worked 4x8 examples, brute-force
  * subset enumeration, invariants, and exact integer matmul cross-checks; for
  * the output stage, hand-worked rounding/saturation cases
  * (tests/golden/epilogue_hand.json), the standard normal CDF table for GELU
- * and the identity GELU(x) - GELU(-x) = x.
+ * and the identity GELU(x) - GELU(-x) = x; for the tile-shared compress,
+ * hand-worked 4x8 examples (tests/golden/tile_hand.json), brute-force
+ * enumeration of the subsets of largest tile mass, the V = 1 reduction to the
+ * per-row rule, and an fp16 case that single-precision sums would decide wrongly.
  */
 #include <math.h>
 #include <stdint.h>
@@ -140,6 +147,66 @@ int oracle_compress(const void *W, int64_t n_out, int64_t k, int dtype, int N, i
                     *byte |= (uint8_t)((p & 0xF) << ((e & 1) ? 4 : 0));
                     ++e;
                 }
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Tile-shared compress, the vector-wise reading of the micro-dense format
+ * (section 4.2: the kept values of a window become a dense tile that regular
+ * MMA fragments consume, the activations being gathered to match).  For a
+ * gather to serve a whole tile of output channels, those channels must keep
+ * the same positions, so rows are taken in tiles of V consecutive rows (the
+ * last tile may be shorter) and, in every tile and group of M positions:
+ *   score(p) = sum over the tile's rows of |w[r][gM + p]|,
+ *   p is kept iff fewer than N positions q of the group precede it in the
+ *   order (score descending, position ascending).
+ * This is the top-N rule of oracle_compress with the tile's column mass as the
+ * magnitude; V = 1 is exactly oracle_compress.  Output uses the same canonical
+ * layout as oracle_compress (every row of a tile carries the same positions).
+ *
+ * Scores are exact.  int8 magnitudes are integers.  fp16 magnitudes are whole
+ * multiples of 2^-24 below 2^16, so a sum of V <= 4096 of them is a multiple of
+ * 2^-24 below 2^28, i.e. an integer below 2^52 in units of 2^-24: exact in
+ * double.  bfloat16 sums can round, so bfloat16 is refused (-3).
+ * Returns 0, -1 for an invalid argument, -3 for an unsupported dtype.
+ */
+int oracle_compress_tile(const void *W, int64_t n_out, int64_t k, int dtype, int N, int M,
+                         int64_t V, void *values, uint8_t *idx) {
+    if (!W || !values || !idx || n_out <= 0 || k <= 0 || M <= 0 || M > 16 || N <= 0 ||
+        N > M || k % M != 0 || dtype < 0 || dtype > 2 || V <= 0 || V > 4096)
+        return -1;
+    if (dtype == OR_BF16) return -3;
+    const size_t es = elem_size(dtype);
+    const int64_t groups = k / M;
+    const int64_t pitch = oracle_idx_pitch(k, N, M);
+    const int64_t tiles = (n_out + V - 1) / V;
+    memset(idx, 0, (size_t)(n_out * pitch));
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < tiles; ++t) {
+        const int64_t r0 = t * V;
+        const int64_t r1 = r0 + V < n_out ? r0 + V : n_out;
+        for (int64_t g = 0; g < groups; ++g) {
+            double score[16];
+            for (int p = 0; p < M; ++p) {
+                score[p] = 0.0;
+                for (int64_t r = r0; r < r1; ++r) score[p] += magnitude(W, dtype, r * k + g * M + p);
+            }
+            int e = 0; /* kept-element counter within the group */
+            for (int p = 0; p < M; ++p) {
+                int ahead = 0;
+                for (int q = 0; q < M; ++q)
+                    if (score[q] > score[p] || (score[q] == score[p] && q < p)) ++ahead;
+                if (ahead >= N) continue;
+                for (int64_t r = r0; r < r1; ++r) {
+                    const int64_t el = g * N + e; /* element index within the row */
+                    memcpy((char *)values + (size_t)(r * groups * N + el) * es,
+                           (const char *)W + (size_t)(r * k + g * M + p) * es, es);
+                    idx[r * pitch + el / 2] |= (uint8_t)((p & 0xF) << ((el & 1) ? 4 : 0));
+                }
+                ++e;
             }
         }
     }
