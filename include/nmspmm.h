@@ -191,6 +191,52 @@ nm_status nm_spmm_ex(const nm_handle* h, const void* X_dev, int64_t T, void* Y_d
                      const nm_epilogue* ep, void* stream);
 
 /*
+ * nm_compress_tile -- prune and pack one weight with a pattern shared by each
+ * tile of 128 consecutive output channels (the vector-wise reading of the
+ * paper's section 4.2: kept values become dense MMA tiles and the activations
+ * are gathered to match, which needs one set of kept positions per tile of
+ * channels).
+ *
+ * For every tile of rows [128t, 128t + 128) (the last may be shorter) and
+ * every group g of M consecutive k positions, the score of position p is
+ * sum over the tile's rows of |W[n][gM + p]|, computed exactly; the N
+ * positions of largest score are kept, ties to the lower position, and every
+ * row of the tile keeps them.  The handle holds the canonical format (exactly
+ * as nm_compress lays it out, nm_export) and a dense operand image over the
+ * kept k only (K' = k * N / M per row) plus the tile's kept k list, which
+ * nm_spmm_gather uses to gather rows of the activation.
+ *
+ * Arguments as nm_compress, except:
+ *   dt      NM_INT8 or NM_FP16 (scores of bfloat16 weights are not exact in
+ *           any fixed-width sum: NM_ERR_UNSUPPORTED);
+ *   (N, M)  one of (1,4), (2,4), (2,8), (4,8), or N == M with M in {4, 8}.
+ * nm_recompress, nm_decompress, nm_export, nm_query and nm_destroy accept the
+ * handle; nm_spmm, nm_spmm_ex and nm_spmm_noalloc reject it (NM_ERR_INVALID):
+ * its product is nm_spmm_gather.
+ */
+nm_status nm_compress_tile(const void* W_dev, int64_t n_out, int64_t k, nm_dtype dt, int N, int M,
+                           void* stream, nm_handle** out);
+
+/*
+ * nm_spmm_gather -- Y = X . Wm^T for a handle made by nm_compress_tile, with
+ * the activation given feature-major: Xt_dev [k][ldx] holds X[t][kk] at
+ * Xt_dev[kk * ldx + t].  Per 128-channel tile the kernel gathers the kept rows
+ * of Xt (tensor-memory-access gathers of four rows per copy) into a dense
+ * operand and runs dense tensor-core MMAs over K' = k * N / M only, so both
+ * the MMA work and the activation bytes read per tile shrink by N / M.
+ *
+ * Xt_dev    16-byte aligned; ldx >= T and ldx * sizeof(dtype) a multiple of
+ *           16 bytes (else NM_ERR_INVALID).  Columns t >= T are not read.
+ * Y_dev     [T][n_out], 16-byte aligned, not overlapping Xt; element type and
+ *           rounding exactly as nm_spmm (INT8: int32, or float32 with scale;
+ *           FP16: fp16 from the fp32 accumulator).
+ * scale_dev float32 [n_out] or NULL.
+ * T         >= 0; T == 0 is a no-op.  Never synchronises.
+ */
+nm_status nm_spmm_gather(const nm_handle* h, const void* Xt_dev, int64_t ldx, int64_t T, void* Y_dev,
+                         const float* scale_dev, void* stream);
+
+/*
  * nm_decompress -- write the masked dense weight Wm [n_out][k] (dtype of the
  * handle) decoded from the packed operand image the SpMM kernel reads, so the
  * image can be checked against the top-N rule.  W_dev_out 16-byte aligned.

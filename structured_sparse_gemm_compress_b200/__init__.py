@@ -24,7 +24,8 @@ _TORCH_DT = {torch.int8: NM_INT8, torch.float16: NM_FP16, torch.bfloat16: NM_BF1
 _ELEM = {NM_INT8: torch.int8, NM_FP16: torch.float16, NM_BF16: torch.bfloat16}
 
 # Every symbol include/nmspmm.h declares.
-EXPORTS = ("nm_compress", "nm_recompress", "nm_spmm", "nm_spmm_ex", "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
+EXPORTS = ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_ex", "nm_spmm_gather",
+           "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
            "nm_device_status", "nm_destroy", "nm_last_error", "nm_version", "nm_test_spmm_skip_stage")
 
 
@@ -47,6 +48,8 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
         L.nm_compress.argtypes = [vp, i64, i64, i32, i32, i32, vp, ctypes.POINTER(vp)]
+        L.nm_compress_tile.argtypes = [vp, i64, i64, i32, i32, i32, vp, ctypes.POINTER(vp)]
+        L.nm_spmm_gather.argtypes = [vp, vp, i64, i64, vp, vp, vp]
         L.nm_recompress.argtypes = [vp, vp, vp]
         L.nm_spmm.argtypes = [vp, vp, i64, vp, vp, vp]
         L.nm_spmm_noalloc.argtypes = [vp, vp, i64, vp, vp, vp]
@@ -62,8 +65,9 @@ def lib() -> ctypes.CDLL:
         L.nm_destroy.restype = None
         L.nm_last_error.restype = ctypes.c_char_p
         L.nm_version.restype = ctypes.c_char_p
-        for name in ("nm_compress", "nm_recompress", "nm_spmm", "nm_spmm_noalloc", "nm_test_spmm_skip_stage", "nm_decompress", "nm_export",
-                     "nm_export_sizes", "nm_query", "nm_device_status"):
+        for name in ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_gather", "nm_spmm_noalloc",
+                     "nm_test_spmm_skip_stage", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
+                     "nm_device_status"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -89,9 +93,10 @@ def _ptr(t: torch.Tensor | None) -> int | None:
 class NMHandle:
     """One compressed weight (owns the library handle and its device memory)."""
 
-    def __init__(self, raw: int, n_out: int, k: int, N: int, M: int, dt: int):
+    def __init__(self, raw: int, n_out: int, k: int, N: int, M: int, dt: int, tile: bool = False):
         self._raw = ctypes.c_void_p(raw)
         self.n_out, self.k, self.N, self.M, self.dt = n_out, k, N, M, dt
+        self.tile = tile  # one pattern per 128-channel tile (nm_compress_tile)
 
     @property
     def raw(self) -> ctypes.c_void_p:
@@ -128,6 +133,20 @@ def nm_compress(W: torch.Tensor, N: int, M: int, stream=None) -> NMHandle:
     return NMHandle(out.value, n_out, k, N, M, _TORCH_DT[W.dtype])
 
 
+def nm_compress_tile(W: torch.Tensor, N: int, M: int, stream=None) -> NMHandle:
+    """Prune W [n_out, k] (int8 / fp16, on the GPU) to N:M with one pattern per
+    128-row tile (largest column mass) and pack it for ``nm_spmm_gather``."""
+    if not W.is_cuda:
+        raise ValueError("W must be a CUDA tensor")
+    if W.dtype not in _TORCH_DT:
+        raise ValueError(f"unsupported dtype {W.dtype}")
+    W = W.contiguous()
+    n_out, k = W.shape
+    out = ctypes.c_void_p()
+    _check(lib().nm_compress_tile(_ptr(W), n_out, k, _TORCH_DT[W.dtype], N, M, _stream(stream), ctypes.byref(out)))
+    return NMHandle(out.value, n_out, k, N, M, _TORCH_DT[W.dtype], tile=True)
+
+
 def nm_recompress(h: NMHandle, W: torch.Tensor, stream=None) -> NMHandle:
     """Re-prune and re-pack a new weight of the same shape/dtype into ``h`` (no allocation)."""
     if not W.is_cuda or W.dtype != h.dtype or tuple(W.shape) != (h.n_out, h.k) or not W.is_contiguous():
@@ -156,6 +175,26 @@ def nm_spmm(h: NMHandle, X: torch.Tensor, Y: torch.Tensor | None = None, scale: 
     if scale is not None and (scale.dtype != torch.float32 or scale.numel() != h.n_out or not scale.is_cuda):
         raise ValueError("scale must be a CUDA float32 tensor of n_out elements")
     _check(lib().nm_spmm(h.raw, _ptr(X), T, _ptr(Y), _ptr(scale), _stream(stream)))
+    return Y
+
+
+def nm_spmm_gather(h: NMHandle, Xt: torch.Tensor, T: int | None = None, Y: torch.Tensor | None = None,
+                   scale: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = X @ Wm^T for a tile-shared handle, X given feature-major as
+    ``Xt`` [k, ldx] (``Xt[kk, t] = X[t, kk]``, rows contiguous, ldx = the row
+    stride); T defaults to ``Xt.shape[1]``."""
+    if Xt.dtype != h.dtype or not Xt.is_cuda or Xt.dim() != 2 or Xt.shape[0] != h.k or Xt.stride(1) != 1:
+        raise ValueError("Xt must be a CUDA [k, T] tensor of the handle's dtype with contiguous rows")
+    T = Xt.shape[1] if T is None else int(T)
+    want = out_dtype(h, scale is not None)
+    if Y is None:
+        Y = torch.empty((T, h.n_out), dtype=want, device=Xt.device)
+    elif Y.dtype != want or tuple(Y.shape) != (T, h.n_out) or not Y.is_contiguous():
+        raise ValueError(f"Y must be a contiguous [{T}, {h.n_out}] {want} tensor")
+    if scale is not None and (scale.dtype != torch.float32 or scale.numel() != h.n_out or not scale.is_cuda):
+        raise ValueError("scale must be a CUDA float32 tensor of n_out elements")
+    ldx = Xt.stride(0) if Xt.shape[0] > 1 else Xt.shape[1]
+    _check(lib().nm_spmm_gather(h.raw, _ptr(Xt), ldx, T, _ptr(Y), _ptr(scale), _stream(stream)))
     return Y
 
 

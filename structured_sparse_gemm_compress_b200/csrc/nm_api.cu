@@ -100,6 +100,36 @@ nm_status make_x_map(nm_handle* h, const void* X, int64_t T, int bn) {  // bn = 
   h->tm_x = X;
   h->tm_T = T;
   h->tm_bn = bn;
+  h->tm_ld = -1;
+  return NM_OK;
+}
+
+// Feature-major activation Xt [k][ldx] (only the first T columns exist) as a
+// 2-D tensor whose rows are features: box = one row x 128 bytes of tokens,
+// 128-byte swizzle, so a four-row gather lands as four rows of the MN-major
+// operand layout; tokens beyond T read as zero.
+nm_status make_xt_map(nm_handle* h, const void* Xt, int64_t ldx, int64_t T) {
+  if (h->tm_x == Xt && h->tm_T == T && h->tm_ld == ldx) return NM_OK;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int es = nm::elem_bytes(h->dt);
+  CUtensorMapDataType ty = h->dt == nm::DT_I8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  cuuint64_t dims[2] = {(cuuint64_t)T, (cuuint64_t)h->k};
+  cuuint64_t strides[1] = {(cuuint64_t)(ldx * es)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / es), 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&h->tm, ty, 2, const_cast<void*>(Xt), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    h->tm_x = nullptr;
+    return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for Xt with T=%lld ldx=%lld k=%lld", (int)r,
+                (long long)T, (long long)ldx, (long long)h->k);
+  }
+  h->tm_x = Xt;
+  h->tm_T = T;
+  h->tm_ld = ldx;
+  h->tm_bn = 0;
   return NM_OK;
 }
 
@@ -180,6 +210,27 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
   const int forced_xs = env_int("NMSPMM_FORCE_XS", -1);  // -1 auto, 0 off, 1 on when eligible
   const int forced_grid = env_int("NMSPMM_FORCE_GRID", 0);  // cap on persistent CTAs (tests, sweeps)
   if (forced_grid > 0) sms = std::min(sms, forced_grid);
+  if (h->tile) {
+    // Gather image (streaming kernel only): token tiles of 256 or 128, by the
+    // same waves x (BN + fixed cost) model as below; split-K only when forced.
+    double best = 1e300;
+    for (int bn : {256, 128}) {
+      if (forced_bn && bn != forced_bn) continue;
+      const int64_t tiles = (int64_t)h->n_ct * ((T + bn - 1) / bn);
+      const double cost = (double)((tiles + sms - 1) / sms) * (bn + 140);
+      if (cost < best) {
+        best = cost;
+        p.bn = bn;
+      }
+    }
+    p.n_tt = (int)((T + p.bn - 1) / p.bn);
+    const int splits = std::max(1, std::min(forced_split > 0 ? forced_split : 1, h->n_kb));
+    p.kb_per_split = (h->n_kb + splits - 1) / splits;
+    p.splits = (h->n_kb + p.kb_per_split - 1) / p.kb_per_split;
+    p.units = (int)((int64_t)h->n_ct * p.n_tt * p.splits);
+    p.grid = std::min(p.units, sms);
+    return p;
+  }
   // CTA-pair mode (M = 256 per MMA, one issuing thread per two SMs): whenever
   // there are enough 256-channel x BN-token tiles to occupy every resident pair.
   const int forced_pair = env_int("NMSPMM_FORCE_PAIR", -1);  // -1 auto, 0 off, 1 on
@@ -288,11 +339,17 @@ int out_elem_bytes(const nm_handle* h, const EpiReq* ep) {
   return h->dt == nm::DT_I8 ? 4 : 2;
 }
 
+nm_status reject_tile(const nm_handle* h) {
+  if (h->tile) return fail(NM_ERR_INVALID, "the handle was made by nm_compress_tile: its product is nm_spmm_gather");
+  return NM_OK;
+}
+
 nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, const float* scale, void* stream,
                     int inject_skip, unsigned long long timeout_ns, const EpiReq* ep = nullptr) {
   g_err.clear();
   nm_status st = check_handle(hc);
   if (st != NM_OK) return st;
+  if ((st = reject_tile(hc)) != NM_OK) return st;
   nm_handle* h = const_cast<nm_handle*>(hc);  // only caches (tensor map, workspace) change
   if (T < 0) return fail(NM_ERR_INVALID, "T must be >= 0 (got %lld)", (long long)T);
   if (T == 0) return NM_OK;
@@ -480,7 +537,8 @@ nm_status nm_recompress(nm_handle* h, const void* W_dev, void* stream) {
   if (st != NM_OK) return st;
   if (!W_dev) return fail(NM_ERR_INVALID, "null W");
   if (!aligned(W_dev, (size_t)nm::elem_bytes(h->dt))) return fail(NM_ERR_INVALID, "W is not element aligned");
-  cudaError_t e = nm::launch_compress(h, W_dev, (cudaStream_t)stream);
+  cudaError_t e = h->tile ? nm::launch_compress_tile(h, W_dev, (cudaStream_t)stream)
+                          : nm::launch_compress(h, W_dev, (cudaStream_t)stream);
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch compress kernel");
 }
 
@@ -528,6 +586,149 @@ nm_status nm_test_spmm_skip_stage(const nm_handle* h, const void* X_dev, int64_t
                                   const float* scale_dev, void* stream, int skip_stage, int64_t timeout_ns) {
   if (timeout_ns <= 0 || timeout_ns > 2000000000ll) return fail(NM_ERR_INVALID, "timeout must be in (0, 2 s]");
   return spmm_impl(h, X_dev, T, Y_dev, scale_dev, stream, skip_stage, (unsigned long long)timeout_ns);
+}
+
+nm_status nm_compress_tile(const void* W_dev, int64_t n_out, int64_t k, nm_dtype dt, int N, int M, void* stream,
+                           nm_handle** out) {
+  g_err.clear();
+  if (!out) return fail(NM_ERR_INVALID, "null output handle pointer");
+  *out = nullptr;
+  if (!W_dev) return fail(NM_ERR_INVALID, "null W");
+  if ((int)dt < 0 || (int)dt > 2) return fail(NM_ERR_INVALID, "unknown dtype %d", (int)dt);
+  if (dt == NM_BF16)
+    return fail(NM_ERR_UNSUPPORTED, "tile-shared patterns need exact column sums: INT8 and FP16 only");
+  if (n_out <= 0 || k <= 0) return fail(NM_ERR_INVALID, "n_out and k must be positive");
+  if (n_out > (1 << 24) || k > (1 << 24)) return fail(NM_ERR_UNSUPPORTED, "n_out and k are limited to 2^24");
+  if (dt == NM_INT8 && k > (1 << 17))
+    return fail(NM_ERR_UNSUPPORTED, "INT8 k is limited to 2^17 (int32 accumulation must not overflow)");
+  if (M <= 0 || N <= 0 || N > M) return fail(NM_ERR_INVALID, "bad N:M %d:%d", N, M);
+  const bool ok = (N == 1 && M == 4) || (N == 2 && M == 4) || (N == 2 && M == 8) || (N == 4 && M == 8) ||
+                  (N == M && (M == 4 || M == 8));
+  if (!ok) return fail(NM_ERR_UNSUPPORTED, "N:M %d:%d is not supported", N, M);
+  if (k % M != 0) return fail(NM_ERR_INVALID, "k=%lld is not a multiple of M=%d", (long long)k, M);
+  const int es = nm::elem_bytes((int)dt);
+  if (!aligned(W_dev, (size_t)es)) return fail(NM_ERR_INVALID, "W is not element aligned");
+
+  nm_handle* h = new (std::nothrow) nm_handle();
+  if (!h) return fail(NM_ERR_OOM, "host allocation failed");
+  cudaGetDevice(&h->device);
+  h->n_out = n_out;
+  h->k = k;
+  h->N = N;
+  h->M = M;
+  h->dt = (int)dt;
+  h->tile = 1;
+  h->img = nm::IMG_GATHER;
+  h->kp = (k / M) * N;
+  const int KBG = nm::gather_kblock_elems(h->dt);
+  h->n_kb = (int)((h->kp + KBG - 1) / KBG);
+  h->n_ct = (int)((n_out + nm::kRows - 1) / nm::kRows);
+  h->chunk = (size_t)nm::chunk_bytes(h->dt, h->img);
+  h->values_bytes = (size_t)n_out * (size_t)h->kp * es;
+  h->idx_pitch = (h->kp + 1) / 2;
+  h->idx_bytes = (size_t)n_out * (size_t)h->idx_pitch;
+  h->bpack_bytes = (size_t)h->n_ct * h->n_kb * h->chunk;
+  h->kidx_bytes = (size_t)h->n_ct * h->n_kb * KBG * sizeof(int32_t);
+
+  cudaError_t e;
+  nm_status st = NM_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((e = cudaMalloc(&h->d_values, h->values_bytes)) != cudaSuccess) st = cuda_fail(e, "allocate values");
+  else if ((e = cudaMalloc(&h->d_idx, h->idx_bytes)) != cudaSuccess) st = cuda_fail(e, "allocate idx");
+  else if ((e = cudaMalloc(&h->d_bpack, h->bpack_bytes)) != cudaSuccess) st = cuda_fail(e, "allocate packed image");
+  else if ((e = cudaMalloc(&h->d_kidx, h->kidx_bytes)) != cudaSuccess) st = cuda_fail(e, "allocate kept k lists");
+  else if ((e = cudaMalloc(&h->d_err, sizeof(int))) != cudaSuccess) st = cuda_fail(e, "allocate error word");
+  else if ((e = cudaMemsetAsync(h->d_err, 0, sizeof(int), s)) != cudaSuccess) st = cuda_fail(e, "clear error word");
+  else if ((e = cudaMemsetAsync(h->d_kidx, 0, h->kidx_bytes, s)) != cudaSuccess)  // padding slots gather row 0
+    st = cuda_fail(e, "clear kept k lists");
+  else if ((e = nm::launch_compress_tile(h, W_dev, s)) != cudaSuccess)
+    st = cuda_fail(e, "launch compress kernels");
+  else
+    st = make_w_map(h);
+  if (st != NM_OK) {
+    const std::string msg = g_err;
+    nm_destroy(h);
+    g_err = msg;
+    return st;
+  }
+  *out = h;
+  return NM_OK;
+}
+
+nm_status nm_spmm_gather(const nm_handle* hc, const void* Xt, int64_t ldx, int64_t T, void* Y, const float* scale,
+                         void* stream) {
+  g_err.clear();
+  nm_status st = check_handle(hc);
+  if (st != NM_OK) return st;
+  if (!hc->tile) return fail(NM_ERR_INVALID, "nm_spmm_gather needs a handle made by nm_compress_tile");
+  nm_handle* h = const_cast<nm_handle*>(hc);  // only caches (tensor map, workspace) change
+  if (T < 0) return fail(NM_ERR_INVALID, "T must be >= 0 (got %lld)", (long long)T);
+  if (T == 0) return NM_OK;
+  if (!Xt || !Y) return fail(NM_ERR_INVALID, "null Xt or Y");
+  if (T > INT32_MAX) return fail(NM_ERR_UNSUPPORTED, "T above 2^31-1");
+  const int es = nm::elem_bytes(h->dt);
+  if (ldx < T) return fail(NM_ERR_INVALID, "ldx=%lld is below T=%lld", (long long)ldx, (long long)T);
+  if ((ldx * es) % 16 != 0)
+    return fail(NM_ERR_INVALID, "ldx * sizeof(dtype) must be a multiple of 16 bytes (ldx=%lld)", (long long)ldx);
+  if (!aligned(Xt, 16) || !aligned(Y, 16)) return fail(NM_ERR_INVALID, "Xt and Y must be 16-byte aligned");
+  if (scale && !aligned(scale, 4)) return fail(NM_ERR_INVALID, "scale must be 4-byte aligned");
+  const size_t ybytes = (size_t)T * h->n_out * out_elem_bytes(h, nullptr);
+  const size_t xbytes = ((size_t)(h->k - 1) * ldx + T) * es;
+  const uintptr_t xs = (uintptr_t)Xt, ys = (uintptr_t)Y;
+  if (xs < ys + ybytes && ys < xs + xbytes) return fail(NM_ERR_INVALID, "Y overlaps Xt");
+
+  const nm::Plan p = make_plan(h, T, num_sms(h->device), scale != nullptr);
+  st = make_xt_map(h, Xt, ldx, T);
+  if (st != NM_OK) return st;
+  nm::SpmmArgs a{};
+  a.bpack = h->d_bpack;
+  a.Y = Y;
+  a.scale = scale;
+  a.err = h->d_err;
+  a.T = (int)T;
+  a.n_out = (int)h->n_out;
+  a.n_kb = h->n_kb;
+  a.n_ct = h->n_ct;
+  a.n_tt = p.n_tt;
+  a.splits = p.splits;
+  a.kb_per_split = p.kb_per_split;
+  a.units = p.units;
+  a.timeout_ns = 1000000000ull;
+  a.inject_skip = -1;
+  a.w_tma = (h->has_tmw && env_int("NMSPMM_W_BULK", 0) == 0) ? 1 : 0;
+  a.tma_store = 0;
+  a.kidx = h->d_kidx;
+  a.xt = Xt;
+  a.ldx = (long long)ldx;
+  // Gather warps (load/store path) by default: measured faster on B200 than
+  // four-row tensor gathers, whose per-copy cost caps them near 1.3 TB/s.
+  a.gather_tma = env_int("NMSPMM_GATHER_TMA", 0) ? 1 : 0;
+  if (p.splits > 1) {
+    const int tiles = h->n_ct * p.n_tt;
+    const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
+    if (need > h->ws_bytes || tiles > h->cnt_len) {
+      cudaError_t e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) return cuda_fail(e, "synchronise before growing the split-K workspace");
+      cudaFree(h->d_ws);
+      cudaFree(h->d_cnt);
+      h->d_ws = nullptr;
+      h->d_cnt = nullptr;
+      h->ws_bytes = 0;
+      h->cnt_len = 0;
+      const int cl = std::max(tiles, 256);
+      if ((e = cudaMalloc(&h->d_ws, need)) != cudaSuccess) return cuda_fail(e, "allocate split-K workspace");
+      if ((e = cudaMalloc(&h->d_cnt, (size_t)cl * sizeof(int))) != cudaSuccess)
+        return cuda_fail(e, "allocate split-K counters");
+      if ((e = cudaMemset(h->d_cnt, 0, (size_t)cl * sizeof(int))) != cudaSuccess)
+        return cuda_fail(e, "clear split-K counters");
+      h->ws_bytes = need;
+      h->cnt_len = cl;
+    }
+    a.ws = h->d_ws;
+    a.cnt = h->d_cnt;
+  }
+  cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch SpMM kernel");
 }
 
 nm_status nm_decompress(const nm_handle* h, void* W_dev_out, void* stream) {
@@ -594,6 +795,7 @@ nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y
   g_err.clear();
   nm_status st = check_handle(hc);
   if (st != NM_OK) return st;
+  if ((st = reject_tile(hc)) != NM_OK) return st;
   nm_handle* h = const_cast<nm_handle*>(hc);  // only the tensor-map cache (host memory) changes
   void* scratch = nullptr;
   st = noalloc_scratch(h->device, &scratch);  // first call on this device: address lookup
@@ -665,6 +867,7 @@ void nm_destroy(nm_handle* h) {
   cudaFree(h->d_values);
   cudaFree(h->d_idx);
   cudaFree(h->d_bpack);
+  cudaFree(h->d_kidx);
   cudaFree(h->d_err);
   cudaFree(h->d_ws);
   cudaFree(h->d_cnt);

@@ -26,6 +26,11 @@
 //   dense-image chunk (pattern 4:8 and N == M): [ A: two 128 x 128 B swizzled
 //     atoms ] holding the masked dense tile (bytes [128a, 128a+128) of each
 //     row in atom a).
+//   gather-image chunk (handles with one pattern per 128-row tile): [ A: one
+//     128 x 128 B swizzled atom ] holding 128 B of the tile's kept values per
+//     row (128 kept k for INT8, 64 for FP16), i.e. a dense operand over the
+//     kept k only; the tile's kept k list (int32, padded with 0 to whole
+//     k-blocks) names the activation rows each k-block gathers.
 // Rows beyond n_out and k beyond K are zero (metadata nibble 0).
 #pragma once
 #include <cstdint>
@@ -35,7 +40,7 @@
 namespace nm {
 
 enum : int { DT_I8 = 0, DT_F16 = 1, DT_BF16 = 2 };
-enum : int { IMG_SP24 = 0, IMG_DENSE = 1 };
+enum : int { IMG_SP24 = 0, IMG_DENSE = 1, IMG_GATHER = 2 };
 enum : int { OUT_I32 = 0, OUT_F32 = 1, OUT_F16 = 2, OUT_BF16 = 3, OUT_I8 = 4 };  // output element of a launch
 enum : int { ACT_NONE = 0, ACT_GELU = 1 };  // activation of the fused output stage
 
@@ -46,8 +51,10 @@ __host__ __device__ constexpr int kblock_elems(int dt) { return dt == DT_I8 ? 25
 __host__ __device__ constexpr int elem_bytes(int dt) { return dt == DT_I8 ? 1 : 2; }
 __host__ __device__ constexpr int meta_bytes(int dt) { return dt == DT_I8 ? 4096 : 2048; }
 __host__ __device__ constexpr int chunk_bytes(int dt, int img) {
-  return img == IMG_SP24 ? kAtomBytes + meta_bytes(dt) : 2 * kAtomBytes;
+  return img == IMG_SP24 ? kAtomBytes + meta_bytes(dt) : img == IMG_GATHER ? kAtomBytes : 2 * kAtomBytes;
 }
+// Kept k per k-block of the gather image: one 128-byte row of values.
+__host__ __device__ constexpr int gather_kblock_elems(int dt) { return 128 / elem_bytes(dt); }
 
 // Byte offset of (row r, byte c of the 128-byte row) inside a swizzled atom.
 __host__ __device__ inline uint32_t swz128(uint32_t r, uint32_t c) {
@@ -160,6 +167,18 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Four rows r0..r3 of a 2-D tensor, each one box wide starting at column c0,
+// into four consecutive box-sized rows of shared memory (the tensor map's
+// box must be one row high).
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0,
+                                            int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -269,6 +288,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
   d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset: next 8-row group
   d |= (uint64_t)1u << 46;                 // descriptor version
   d |= (uint64_t)2u << 61;                 // layout: 128-byte swizzle
+  return d;
+}
+
+// Shared-memory descriptor of an MN-major operand with 128-byte swizzle: along
+// MN, 128-byte runs (the swizzle atom's width) lie `mn_block_bytes` apart;
+// along K, rows are 128 B apart and groups of 8 rows 1024 B apart.
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t mn_block_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((mn_block_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next 128-byte MN run
+  d |= (uint64_t)(1024u >> 4) << 32;                        // stride byte offset: next 8 K rows
+  d |= (uint64_t)1u << 46;                                  // descriptor version
+  d |= (uint64_t)2u << 61;                                  // layout: 128-byte swizzle
   return d;
 }
 
@@ -414,6 +446,19 @@ __device__ __forceinline__ void bulk_wait() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA).
+// 16 bytes global -> shared through the load/store path, bypassing L1; bytes
+// of the 16 at or beyond src_bytes (0..16) are written as zero and not read.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {  // all but the newest N groups of this thread have landed
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

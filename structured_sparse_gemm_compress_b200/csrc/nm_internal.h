@@ -23,6 +23,13 @@ struct nm_handle {
   int64_t idx_pitch = 0;
   uint8_t* d_bpack = nullptr; // packed operand image
   size_t bpack_bytes = 0;
+  // one pattern per 128-row tile (nm_compress_tile): the image covers the kept
+  // k only (kp per row) and d_kidx lists, per tile, the kept k of every
+  // k-block slot (n_kb * gather_kblock_elems entries, padded with 0)
+  int tile = 0;
+  int64_t kp = 0;
+  int32_t* d_kidx = nullptr;
+  size_t kidx_bytes = 0;
   int* d_err = nullptr;       // device error word (bounded-wait timeouts)
 
   // split-K workspace (partials + per-tile arrival counters), grown on demand
@@ -34,6 +41,7 @@ struct nm_handle {
   // cached tensor map of the last activation seen
   const void* tm_x = nullptr;
   int64_t tm_T = -1;
+  int64_t tm_ld = -1;     // row pitch (elements) of a feature-major activation map
   int tm_bn = 0;
   alignas(64) CUtensorMap tm;
   // the packed image as a 2-D tensor of 128-byte rows (one box = one chunk)
@@ -89,6 +97,15 @@ struct SpmmArgs {
   const float* bias = nullptr;
   int act = 0;
   float out_scale = 1.0f;
+  // Gather image only: per channel tile, n_kb * gather_kblock_elems kept k
+  // (the activation rows each k-block gathers).
+  const int32_t* kidx = nullptr;
+  // Gather image: the feature-major activation Xt [k][ldx] read by the gather
+  // warps (load/store path), and gather_tma = 1 to gather with four-row tensor
+  // copies from the producer warp instead.
+  const void* xt = nullptr;
+  long long ldx = 0;
+  int gather_tma = 0;
   long long* trace;   // timeline buffer, only written by builds compiled with NM_TRACE
 };
 
@@ -100,6 +117,8 @@ constexpr int kTraceStride = TR_KINDS * kTraceMax;
 
 cudaError_t launch_compress(const nm_handle* h, const void* W, cudaStream_t s);
 cudaError_t launch_decompress(const nm_handle* h, void* Wout, cudaStream_t s);
+// Tile-shared compress (nm_compress_tile): selects each tile's kept k, then packs.
+cudaError_t launch_compress_tile(const nm_handle* h, const void* W, cudaStream_t s);
 // Resident CTA pairs for the pair kernel of this (dtype, image, token tile, output) or <= 0.
 int pair_max_clusters(int dt, int img, int bn, int out);
 cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const CUtensorMap* tmY, const Plan& p,

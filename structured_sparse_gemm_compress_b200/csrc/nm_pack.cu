@@ -467,6 +467,168 @@ __global__ void __launch_bounds__(256) decompress_kernel(const uint8_t* __restri
   for (int c = 0; c < valid; ++c) Wout[r * K + k0 + c] = out[c];
 }
 
+// ------------------------------------------------------------------ tile-shared patterns
+//
+// One pattern per 128-row channel tile (nm_compress_tile): per tile and group
+// of M positions, score(p) = sum over the tile's rows of |w| at p, kept = the N
+// largest scores, ties to the lower position.  Scores are exact integers:
+// |int8| as is, |fp16| in units of 2^-24 (every fp16 magnitude is a whole
+// multiple of 2^-24 below 2^16, so a tile's sum stays below 2^47).
+template <int DT>
+struct TileScore;
+template <>
+struct TileScore<DT_I8> {
+  using S = int;
+  __device__ static S of(int8_t v) { return v < 0 ? -(int)v : (int)v; }
+};
+template <>
+struct TileScore<DT_F16> {
+  using S = long long;
+  __device__ static S of(uint16_t bits) {
+    const int e = (bits >> 10) & 0x1F;
+    const long long m = bits & 0x3FF;
+    return e == 0 ? m : ((m | 0x400) << (e - 1));  // (1.m) * 2^(e-15) = (m | 2^10) * 2^(e-25)
+  }
+};
+
+// Block = 8 row slices x 32 groups; slice s sums rows s, s + 8, ... of the tile,
+// then one thread per group combines the slices and ranks the M positions.
+template <int DT, int N, int M>
+__global__ void __launch_bounds__(256) tile_select_kernel(const typename Elem<DT>::T* __restrict__ W, int64_t n_out,
+                                                          int64_t K, int64_t gblocks, int32_t* __restrict__ kidx,
+                                                          int64_t kidx_pitch) {
+  using S = typename TileScore<DT>::S;
+  constexpr int G = 32, SL = 8;
+  __shared__ S part[SL][G][M];
+  const int gl = threadIdx.x & 31, sl = threadIdx.x >> 5;
+  const int64_t ct = blockIdx.x / gblocks;
+  const int64_t g = (blockIdx.x - ct * gblocks) * G + gl;
+  const int64_t groups = K / M;
+  S acc[M];
+#pragma unroll
+  for (int p = 0; p < M; ++p) acc[p] = 0;
+  if (g < groups) {
+#pragma unroll 4
+    for (int i = sl; i < kRows; i += SL) {
+      const int64_t r = ct * kRows + i;
+      if (r >= n_out) break;
+      const typename Elem<DT>::T* src = W + r * K + g * M;
+#pragma unroll
+      for (int p = 0; p < M; ++p) acc[p] += TileScore<DT>::of(src[p]);
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < M; ++p) part[sl][gl][p] = acc[p];
+  __syncthreads();
+  if (sl != 0 || g >= groups) return;
+  S sc[M];
+#pragma unroll
+  for (int p = 0; p < M; ++p) {
+    S t = 0;
+#pragma unroll
+    for (int q = 0; q < SL; ++q) t += part[q][gl][p];
+    sc[p] = t;
+  }
+  int e = 0;
+#pragma unroll
+  for (int p = 0; p < M; ++p) {
+    int ahead = 0;
+#pragma unroll
+    for (int q = 0; q < M; ++q) ahead += (sc[q] > sc[p] || (sc[q] == sc[p] && q < p)) ? 1 : 0;
+    if (ahead < N) kidx[ct * kidx_pitch + g * N + e++] = (int32_t)(g * M + p);
+  }
+}
+
+// One thread per (row, 16 consecutive kept slots): gathers the kept values
+// through the tile's kept k list and writes the canonical format (rows < n_out,
+// slots < kp) and the gather image (zero beyond them).
+template <int DT>
+__global__ void __launch_bounds__(256) tile_pack_kernel(const typename Elem<DT>::T* __restrict__ W, int64_t n_out,
+                                                        int64_t K, int64_t kp, int M, int n_kb,
+                                                        const int32_t* __restrict__ kidx, int64_t kidx_pitch,
+                                                        typename Elem<DT>::T* __restrict__ values,
+                                                        uint8_t* __restrict__ idx, int64_t idx_pitch,
+                                                        uint8_t* __restrict__ bpack, int64_t total_units) {
+  using T = typename Elem<DT>::T;
+  constexpr int KBG = gather_kblock_elems(DT);
+  constexpr int ES = elem_bytes(DT);
+  const int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (unit >= total_units) return;
+  const int64_t units_per_row = (int64_t)n_kb * (KBG / 16);
+  const int64_t r = unit / units_per_row;
+  const int64_t e0 = (unit - r * units_per_row) * 16;
+  const int64_t ct = r / kRows;
+  int32_t kk[16];
+  const int4* kl = reinterpret_cast<const int4*>(kidx + ct * kidx_pitch + e0);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int4 v = __ldg(kl + q);
+    kk[4 * q] = v.x; kk[4 * q + 1] = v.y; kk[4 * q + 2] = v.z; kk[4 * q + 3] = v.w;
+  }
+  const bool row_ok = r < n_out;
+  T v[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = (row_ok && e0 + j < kp) ? W[r * K + kk[j]] : (T)0;
+
+  if (row_ok) {  // canonical format
+    const int cnt = (int)(kp - e0 < 16 ? kp - e0 : 16);
+    uint32_t nib[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < cnt) nib[j / 8] |= (uint32_t)(kk[j] % M) << (4 * (j % 8));
+    if (cnt == 16) {
+      const uint4 lo = pack16<T>(v);
+      uint32_t vw[8] = {lo.x, lo.y, lo.z, lo.w, 0u, 0u, 0u, 0u};
+      if constexpr (ES == 2) {
+        const uint4 hi = pack16<T>(v + 8);
+        vw[4] = hi.x; vw[5] = hi.y; vw[6] = hi.z; vw[7] = hi.w;
+      }
+      store_bytes(reinterpret_cast<uint8_t*>(values + r * kp + e0), vw, 16 * ES);
+      store_bytes(idx + r * idx_pitch + e0 / 2, nib, 8);
+    } else {
+      for (int j = 0; j < cnt; ++j) values[r * kp + e0 + j] = v[j];
+      for (int b = 0; b < (cnt + 1) / 2; ++b) idx[r * idx_pitch + e0 / 2 + b] = (uint8_t)(nib[b / 4] >> (8 * (b % 4)));
+    }
+  }
+
+  // gather image: 16 slots = 16 * ES bytes of the tile row's 128-byte k-block row
+  const uint32_t rr = (uint32_t)(r % kRows);
+  const int kb = (int)(e0 / KBG);
+  const uint32_t byte0 = (uint32_t)(e0 % KBG) * ES;
+  uint8_t* chunk = bpack + ((size_t)ct * n_kb + kb) * (size_t)chunk_bytes(DT, IMG_GATHER);
+#pragma unroll
+  for (int h = 0; h < ES; ++h)
+    *reinterpret_cast<uint4*>(chunk + swz128(rr, byte0 + 16u * h)) = pack16<T>(v + h * (16 / ES));
+}
+
+// Masked dense weight from the gather image and the kept k list (Wout zeroed first).
+template <int DT>
+__global__ void __launch_bounds__(256) tile_decompress_kernel(const uint8_t* __restrict__ bpack, int64_t n_out,
+                                                              int64_t K, int64_t kp, int n_kb,
+                                                              const int32_t* __restrict__ kidx, int64_t kidx_pitch,
+                                                              typename Elem<DT>::T* __restrict__ Wout,
+                                                              int64_t total_units) {
+  using T = typename Elem<DT>::T;
+  constexpr int KBG = gather_kblock_elems(DT);
+  constexpr int ES = elem_bytes(DT);
+  const int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (unit >= total_units) return;
+  const int64_t units_per_row = (kp + 15) / 16;
+  const int64_t r = unit / units_per_row;
+  const int64_t e0 = (unit - r * units_per_row) * 16;
+  const int64_t ct = r / kRows;
+  const uint32_t rr = (uint32_t)(r % kRows);
+  const int kb = (int)(e0 / KBG);
+  const uint32_t byte0 = (uint32_t)(e0 % KBG) * ES;
+  const uint8_t* chunk = bpack + ((size_t)ct * n_kb + kb) * (size_t)chunk_bytes(DT, IMG_GATHER);
+  T v[16];
+#pragma unroll
+  for (int h = 0; h < ES; ++h)
+    unpack16<T>(*reinterpret_cast<const uint4*>(chunk + swz128(rr, byte0 + 16u * h)), v + h * (16 / ES));
+  const int cnt = (int)(kp - e0 < 16 ? kp - e0 : 16);
+  for (int j = 0; j < cnt; ++j) Wout[r * K + kidx[ct * kidx_pitch + e0 + j]] = v[j];
+}
+
 }  // namespace
 
 template <int DT, int N, int M>
@@ -503,7 +665,67 @@ cudaError_t launch_compress(const nm_handle* h, const void* W, cudaStream_t s) {
   }
 }
 
+template <int DT, int N, int M>
+static void launch_tile_select_t(const nm_handle* h, const void* W, cudaStream_t s) {
+  using T = typename Elem<DT>::T;
+  const int64_t groups = h->k / M;
+  const int64_t gblocks = (groups + 31) / 32;
+  const int64_t kidx_pitch = (int64_t)h->n_kb * gather_kblock_elems(DT);
+  tile_select_kernel<DT, N, M><<<(unsigned)(gblocks * h->n_ct), 256, 0, s>>>((const T*)W, h->n_out, h->k, gblocks,
+                                                                              h->d_kidx, kidx_pitch);
+}
+
+template <int DT>
+static cudaError_t launch_compress_tile_dt(const nm_handle* h, const void* W, cudaStream_t s) {
+  using T = typename Elem<DT>::T;
+  switch (h->N * 16 + h->M) {
+    case 1 * 16 + 4: launch_tile_select_t<DT, 1, 4>(h, W, s); break;
+    case 2 * 16 + 4: launch_tile_select_t<DT, 2, 4>(h, W, s); break;
+    case 2 * 16 + 8: launch_tile_select_t<DT, 2, 8>(h, W, s); break;
+    case 4 * 16 + 8: launch_tile_select_t<DT, 4, 8>(h, W, s); break;
+    case 4 * 16 + 4: launch_tile_select_t<DT, 4, 4>(h, W, s); break;
+    case 8 * 16 + 8: launch_tile_select_t<DT, 8, 8>(h, W, s); break;
+    default: return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  constexpr int KBG = gather_kblock_elems(DT);
+  const int64_t kidx_pitch = (int64_t)h->n_kb * KBG;
+  const int64_t total = (int64_t)h->n_ct * kRows * ((int64_t)h->n_kb * (KBG / 16));
+  const unsigned blocks = (unsigned)((total + 255) / 256);
+  tile_pack_kernel<DT><<<blocks, 256, 0, s>>>((const T*)W, h->n_out, h->k, h->kp, h->M, h->n_kb, h->d_kidx,
+                                             kidx_pitch, (T*)h->d_values, h->d_idx, h->idx_pitch, h->d_bpack, total);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compress_tile(const nm_handle* h, const void* W, cudaStream_t s) {
+  switch (h->dt) {
+    case DT_I8: return launch_compress_tile_dt<DT_I8>(h, W, s);
+    case DT_F16: return launch_compress_tile_dt<DT_F16>(h, W, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int DT>
+static cudaError_t launch_tile_decompress_t(const nm_handle* h, void* Wout, cudaStream_t s) {
+  using T = typename Elem<DT>::T;
+  cudaError_t e = cudaMemsetAsync(Wout, 0, (size_t)h->n_out * (size_t)h->k * elem_bytes(DT), s);
+  if (e != cudaSuccess) return e;
+  const int64_t total = h->n_out * ((h->kp + 15) / 16);
+  const int64_t kidx_pitch = (int64_t)h->n_kb * gather_kblock_elems(DT);
+  tile_decompress_kernel<DT><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+      h->d_bpack, h->n_out, h->k, h->kp, h->n_kb, h->d_kidx, kidx_pitch, (T*)Wout, total);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decompress(const nm_handle* h, void* Wout, cudaStream_t s) {
+  if (h->tile) {
+    switch (h->dt) {
+      case DT_I8: return launch_tile_decompress_t<DT_I8>(h, Wout, s);
+      case DT_F16: return launch_tile_decompress_t<DT_F16>(h, Wout, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   const int64_t total = h->n_out * ((h->k + 15) / 16);
   const int threads = 256;
   const unsigned blocks = (unsigned)((total + threads - 1) / threads);

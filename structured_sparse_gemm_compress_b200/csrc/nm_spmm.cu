@@ -54,6 +54,9 @@ constexpr int out_bytes(int out) { return ((out & 3) == OUT_I32 || (out & 3) == 
 // Epilogue warps and CTA size of a kernel with output code OUT.
 constexpr int epi_warps(int out) { return 4 * epw_for((out & kOutEpi) != 0); }
 constexpr int cta_threads(int out) { return 64 + 32 * epi_warps(out); }
+// Gather image: warps that gather the kept activation rows (after the epilogue warps).
+constexpr int kGatherWarps = 8;
+constexpr int kernel_threads(int img, int out) { return cta_threads(out) + (img == IMG_GATHER ? 32 * kGatherWarps : 0); }
 
 // Kernel configuration.  XKB = 0: streaming mode, every stage carries a packed
 // weight chunk and the matching X boxes.  XKB > 0: X-stationary mode, the
@@ -61,17 +64,26 @@ constexpr int cta_threads(int out) { return 64 + 32 * epi_warps(out); }
 // memory while the CTA walks the channel tiles of its range; stages carry only
 // packed weight chunks, so X is read from L2 once per token tile instead of
 // once per 128-channel tile.
+//
+// IMG_GATHER (one pattern per channel tile): the stage's A is one 128-byte atom
+// of kept values (KB = 128 / sizeof(elem) kept k), and B is gathered from the
+// feature-major activation Xt [k][T]: the KB kept rows of the tile, BN tokens
+// each, land MN-major (token-contiguous 128-byte runs, 128-byte swizzle) in NB
+// runs of BN tokens, run j holding tokens [j*128/es, (j+1)*128/es).
 template <int DT, int IMG, int BN, int OUT, int XKB>
 struct Cfg {
   static constexpr bool SP = IMG == IMG_SP24;
+  static constexpr bool GA = IMG == IMG_GATHER;
   static constexpr bool XS = XKB > 0;
-  static constexpr int KB = kblock_elems(DT);
+  static constexpr int KB = GA ? gather_kblock_elems(DT) : kblock_elems(DT);
   static constexpr int CHUNK = chunk_bytes(DT, IMG);
-  static constexpr int B_BOX = BN * 128;            // one 128-byte-wide box of X rows
-  static constexpr int B_KBLK = 2 * B_BOX;          // X bytes of one k-block
+  static constexpr int NB = GA ? BN * elem_bytes(DT) / 128 : 0;  // gather: 128-byte token runs per row
+  static constexpr int B_BOX = GA ? KB * 128 : BN * 128;  // one 128-byte-wide box of X (gather: all KB rows of one run)
+  static constexpr int B_KBLK = GA ? NB * B_BOX : 2 * B_BOX;  // X bytes of one k-block
   static constexpr int STAGE = XS ? CHUNK : CHUNK + B_KBLK;  // multiple of 1024
   static constexpr int X_BYTES = XKB * B_KBLK;      // resident X region (X-stationary mode)
-  static constexpr int MMAS = SP ? 4 : 8;           // MMAs per stage (each 32 B of A per row)
+  static constexpr int MMAS = (SP || GA) ? 4 : 8;   // MMAs per stage (each 32 B of A per row)
+  static_assert(!GA || (!XS && NB >= 1 && BN * elem_bytes(DT) % 128 == 0), "gather tiles are whole 128-byte runs");
   static constexpr int E_COLS = SP ? (DT == DT_I8 ? 8 : 4) : 0;
   static constexpr int E_COL0 = 2 * BN;             // metadata slots after the two accumulators
   static constexpr int COLS_NEEDED = 2 * BN + 2 * E_COLS;
@@ -79,7 +91,7 @@ struct Cfg {
                                    : COLS_NEEDED <= 256 ? 256 : 512;
   // epilogue: each warp owns BN/epw token columns of its lane quarter, in chunks of CH
   static constexpr int EPI_WARPS = epi_warps(OUT);
-  static constexpr int THREADS = cta_threads(OUT);
+  static constexpr int THREADS = kernel_threads(IMG, OUT);
   static constexpr int WCOLS = BN / (EPI_WARPS / 4);
   // chunks of 32 columns, or one chunk of the whole run when it is not a multiple of 32
   static constexpr int CH = (WCOLS % 32 == 0) ? 32 : (WCOLS % 8 == 0 && WCOLS <= 96) ? WCOLS : 8;
@@ -101,11 +113,13 @@ struct Cfg {
   static_assert(WCOLS % CH == 0 && CH % 8 == 0, "epilogue chunking");
 };
 
-// Instruction descriptor: A K-major (sparse or dense), B K-major, M = 128.
-template <int DT, bool SP, int BN, int M_MMA = 128>
+// Instruction descriptor: A K-major (sparse or dense), B K-major (MN-major
+// when B_MN), M = 128.
+template <int DT, bool SP, int BN, int M_MMA = 128, bool B_MN = false>
 __host__ __device__ constexpr uint32_t make_idesc() {
   uint32_t d = 0;
   if (SP) d |= 1u << 2;                    // sparse A
+  if (B_MN) d |= 1u << 16;                 // B MN-major (token-contiguous)
   if (DT == DT_I8) {
     d |= 2u << 4;                          // D: s32
     d |= 1u << 7;                          // A: signed 8-bit
@@ -348,7 +362,7 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]) {
 }
 
 template <int DT, int IMG, int BN, int OUT, int XKB>
-__global__ void __launch_bounds__(cta_threads(OUT), 1)
+__global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                 const __grid_constant__ CUtensorMap tmW, const SpmmArgs a) {
   using C = Cfg<DT, IMG, BN, OUT, XKB>;
@@ -376,8 +390,10 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    // gather image with gather warps: the producer's arrive plus one per gather warp
+    const uint32_t full_count = (C::GA && !a.gather_tma) ? 1u + kGatherWarps : 1u;
     for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(&full_bar[i], 1);
+      mbar_init(&full_bar[i], full_count);
       mbar_init(&empty_bar[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -447,6 +463,13 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
           cur_tt = w.tt;
         }
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++seq) {
+          // gather image: lanes 0 .. KB/4-1 each fetch four of the k-block's
+          // kept rows (read before the wait so the load overlaps it)
+          int4 grow = make_int4(0, 0, 0, 0);
+          if constexpr (C::GA) {
+            if (a.gather_tma && lane < C::KB / 4)
+              grow = __ldg(reinterpret_cast<const int4*>(a.kidx + ((size_t)w.ct * a.n_kb + kb) * C::KB) + lane);
+          }
           if (!mbar_wait_warp(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
             if (issuer) give_up(1);
             ok = false;
@@ -457,15 +480,26 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
             uint8_t* st = smem + (size_t)stage * C::STAGE;
             const int wrow = (w.ct * a.n_kb + kb) * (C::CHUNK / 128);
             if (issuer) {
-              mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)C::STAGE);
+              // bytes the tensor copies bring (gather warps signal their part by arriving)
+              const uint32_t tx = (C::GA && !a.gather_tma) ? (uint32_t)C::CHUNK : (uint32_t)C::STAGE;
+              mbar_arrive_expect_tx(&full_bar[stage], tx);
               if (a.w_tma)  // the packed image as rows of 128 bytes: one box = one chunk
                 tma_load_2d(st, &tmW, &full_bar[stage], 0, wrow);
               else
                 bulk_load(st, a.bpack + ((size_t)w.ct * a.n_kb + kb) * C::CHUNK, (uint32_t)C::CHUNK,
                           &full_bar[stage]);
-              if constexpr (!XS) {
+              if constexpr (!XS && !C::GA) {
                 tma_load_2d(st + C::CHUNK, &tmX, &full_bar[stage], kb * C::KB, w.tt * BN);
                 tma_load_2d(st + C::CHUNK + C::B_BOX, &tmX, &full_bar[stage], kb * C::KB + C::KB / 2, w.tt * BN);
+              }
+            }
+            if constexpr (C::GA) {
+              __syncwarp();  // the stage's byte count is armed before any gather lands
+              if (a.gather_tma && lane < C::KB / 4) {
+#pragma unroll
+                for (int j = 0; j < C::NB; ++j)
+                  tma_gather4(st + C::CHUNK + j * C::B_BOX + lane * 512, &tmX, &full_bar[stage],
+                              w.tt * BN + j * (128 / elem_bytes(DT)), grow.x, grow.y, grow.z, grow.w);
               }
             }
             armed |= 1u << stage;
@@ -492,7 +526,7 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
     // lane issues the tcgen05 copies, MMAs and commits.
     {
       const bool issuer = elect_one();
-      constexpr uint32_t idesc = make_idesc<DT, SP, BN>();
+      constexpr uint32_t idesc = make_idesc<DT, SP, BN, 128, C::GA>();
       int stage = 0, acc = 0, eslot = 0, cur_tt = -1, mseq = 0, mtile = 0;
       uint32_t phase = 0, acc_phase = 0, xphase = 0;
       bool ok = true;
@@ -537,11 +571,17 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
             }
           }
           // descriptors differ only in the start-address field: build once, add offsets
-          const uint64_t ad0 = sdesc_sw128(a_addr), bd0 = sdesc_sw128(b_addr);
+          const uint64_t ad0 = sdesc_sw128(a_addr);
+          const uint64_t bd0 = C::GA ? sdesc_sw128_mn(b_addr, (uint32_t)C::B_BOX) : sdesc_sw128(b_addr);
 #pragma unroll
           for (int j = 0; j < C::MMAS; ++j) {
             const uint32_t accum = (kb > w.kb0 || j > 0) ? 1u : 0u;
-            if constexpr (SP) {
+            if constexpr (C::GA) {
+              // MMA j: 32 bytes of each A row; the matching 32 / es kept rows of B
+              const uint64_t ad = ad0 + (uint64_t)((32u * j) >> 4);
+              const uint64_t bd = bd0 + (uint64_t)(((uint32_t)j * (32u / elem_bytes(DT)) * 128u) >> 4);
+              if (issuer) tc_mma<KIND>(d_tmem, ad, bd, idesc, accum);
+            } else if constexpr (SP) {
               const uint64_t ad = ad0 + (uint64_t)((32u * j) >> 4);
               const uint64_t bd = bd0 + (uint64_t)(((uint32_t)((j >> 1) * C::B_BOX) + 64u * (j & 1)) >> 4);
               uint32_t e_addr, id2;
@@ -578,6 +618,80 @@ __global__ void __launch_bounds__(cta_threads(OUT), 1)
       // Drain: all tcgen05 work issued by this warp completes before TMEM is freed.
       if (issuer) tc_commit(&drain_bar);
       mbar_wait_warp(&drain_bar, 0, &abort_sh, tmo);
+    }
+  } else if (C::GA && warp >= 2 + C::EPI_WARPS) {
+    // ------------------------------------------------------------ gather warps
+    // Gather image: copy the kept rows of the feature-major activation into the
+    // stage's MN-major operand, 16 bytes per thread and copy (8 threads per
+    // 128-byte token run, so each warp instruction reads four 128-byte rows).
+    // A warp signals a stage LAG stages later, once its own copies of it have
+    // landed (wait_group), after a proxy fence that makes them visible to the
+    // tensor core.  Needs STAGES >= LAG + 2 (a stage is re-filled only after
+    // the MMAs that read it, which need the stages signalled before it).
+    if constexpr (C::GA) {
+      if (!a.gather_tma) {
+        constexpr int ES = elem_bytes(DT);
+        constexpr int RSTEP = 32 * kGatherWarps / 8;  // kept rows per pass
+        constexpr int PASSES = C::KB / RSTEP;
+        constexpr int TOK = 128 / ES;                 // tokens per 128-byte run
+        constexpr int LAG = 2;
+        static_assert(C::KB % RSTEP == 0 && C::STAGES >= LAG + 2, "gather warp schedule");
+        const int gt = threadIdx.x - (64 + 32 * C::EPI_WARPS);
+        const int piece = gt & 7;   // 16-byte piece of a 128-byte run
+        const int rsub = gt >> 3;   // first kept row of this thread
+        const uint8_t* xt = static_cast<const uint8_t*>(a.xt);
+        const size_t pitch = (size_t)a.ldx * ES;
+        int stage = 0, pend = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int u = ur.first; ok && u < ur.end; u += ur.step) {
+          const Unit w = decode_unit(u, a);
+          for (int kb = w.kb0; kb < w.kb1; ++kb) {
+            // kept-row indices, loaded before the wait so their latency overlaps it
+            // (not across the proxy fence below, which would wait for them)
+            int rows[PASSES];
+            const int32_t* kl = a.kidx + ((size_t)w.ct * a.n_kb + kb) * C::KB + rsub;
+#pragma unroll
+            for (int i = 0; i < PASSES; ++i) rows[i] = __ldg(kl + i * RSTEP);
+            if (!mbar_wait_warp(&empty_bar[stage], phase ^ 1u, &abort_sh, tmo)) {
+              if (lane == 0) give_up(1);
+              ok = false;
+              break;
+            }
+            uint8_t* bst = smem + (size_t)stage * C::STAGE + C::CHUNK;
+#pragma unroll
+            for (int j = 0; j < C::NB; ++j) {
+              const int tok0 = w.tt * BN + j * TOK + piece * (16 / ES);
+              const int rem = a.T - tok0;
+              const uint32_t bytes = rem <= 0 ? 0u : rem >= 16 / ES ? 16u : (uint32_t)(rem * ES);
+#pragma unroll
+              for (int i = 0; i < PASSES; ++i) {
+                const int row = rsub + i * RSTEP;
+                const uint8_t* src = bytes ? xt + (size_t)rows[i] * pitch + (size_t)tok0 * ES : xt;
+                cp_async16(bst + j * C::B_BOX + swz128((uint32_t)row, (uint32_t)piece * 16u), src, bytes);
+              }
+            }
+            cp_async_commit();
+            if (pend == LAG) {
+              cp_async_wait<LAG>();  // the k-block issued LAG k-blocks ago has landed
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&full_bar[(stage + C::STAGES - LAG) % C::STAGES]);
+            } else {
+              ++pend;
+            }
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        cp_async_wait<0>();
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0)
+          for (int q = pend; q >= 1; --q) mbar_arrive(&full_bar[(stage + C::STAGES - q) % C::STAGES]);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -1158,9 +1272,25 @@ static cudaError_t launch_bn(const CUtensorMap* tmX, const CUtensorMap* tmY, con
   }
 }
 
+// Gather image: streaming kernel only, fixed output stages with direct stores.
+template <int DT, int OUT>
+static cudaError_t launch_gather(const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
+                                 const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  if constexpr (DT != DT_BF16 && (OUT & kOutEpi) == 0 && (OUT & kOutDirect) != 0) {
+    if (p.pair || p.xkb > 0) return cudaErrorInvalidValue;
+    switch (p.bn) {
+      case 128: return launch_t<DT, IMG_GATHER, 128, OUT, 0>(tmX, tmY, tmW, p, a, s);
+      case 256: return launch_t<DT, IMG_GATHER, 256, OUT, 0>(tmX, tmY, tmW, p, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int DT, int OUT>
 static cudaError_t launch_img(int img, const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
                               const Plan& p, const SpmmArgs& a, cudaStream_t s) {
+  if (img == IMG_GATHER) return launch_gather<DT, OUT>(tmX, tmY, tmW, p, a, s);
   return img == IMG_SP24 ? launch_bn<DT, IMG_SP24, OUT>(tmX, tmY, tmW, p, a, s)
                          : launch_bn<DT, IMG_DENSE, OUT>(tmX, tmY, tmW, p, a, s);
 }
