@@ -234,17 +234,22 @@ def run_reference(args, rank: int) -> None:
 # --------------------------------------------------------------------------- other workloads
 
 
-def roofline_point(l, us: float, pk: dict, out_es: int | None = None, biased: bool = False) -> dict:
+def roofline_point(l, us: float, pk: dict, out_es: int | None = None, biased: bool = False,
+                   gather: bool = False) -> dict:
     """Roofline of one problem: t = max(ops / tensor peak, bytes / HBM peak).
 
     Tensor peaks derive from the measured bf16 dense peak with NVIDIA's nominal
     ratios: INT8 dense = 2 x bf16, FP16/BF16 dense = bf16, 2:4-sparse = 2 x dense
-    (1:4, 2:4, 2:8 run on the sparse pipe; 4:8 and N = M on the dense pipe)."""
+    (1:4, 2:4, 2:8 run on the sparse pipe; 4:8 and N = M on the dense pipe).
+    gather: tile-shared patterns, whose MMAs run on the dense pipe over the kept
+    k only (N/M of the dense-equivalent work)."""
     dense_peak = pk["bf16_tflops"] * (2.0 if l.dtype == inputs.INT8 else 1.0)
     sparse = (l.N, l.M) in ((1, 4), (2, 4), (2, 8))
     tc_peak = dense_peak * (2.0 if sparse else 1.0)
     ops = l.dense_ops()
     t_tc = ops / (tc_peak * 1e12) * 1e6
+    if gather:
+        t_tc = ops * l.N / l.M / (dense_peak * 1e12) * 1e6
     bytes_ = alg_bytes_any(l, out_es, biased)
     t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9) * 1e6
     t_roof = max(t_tc, t_hbm)
@@ -367,6 +372,32 @@ def run_search(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def _graph_us(launch, stream, reps: int = 20) -> float:
+    """Time (us) of one launch: `reps` launches back to back in one CUDA graph,
+    events around the replay, best of three replays."""
+    for _ in range(3):
+        launch(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+        for _ in range(reps):
+            launch(cap)
+    g.replay()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, a.elapsed_time(b) * 1e3 / reps)
+    del g
+    return best
+
+
 def run_config(name: str, args) -> None:
     import structured_sparse_gemm_compress_b200 as nm
 
@@ -384,14 +415,34 @@ def run_config(name: str, args) -> None:
     elif name in ("mixed1", "mixed256"):
         T = 197 if name == "mixed1" else 50432
         ls, desc = inputs.vit_b_mixed(T), f"all 48 ViT-B linears at T={T}, per-layer N:M from {{dense,4:8,2:4,2:8,1:4}}"
+    elif name == "gather":
+        ls, desc = inputs.vit_b_int8(), ("ViT-B/16 INT8 linear set, batch 64 (T=12608), N:M in {1:4,2:4,2:8,4:8} with one "
+                                         "pattern per 128-channel tile, activation feature-major, gather SpMM")
+    elif name == "gatherl":
+        ls, desc = inputs.vit_l_fp16(patterns=("1:4", "2:4", "2:8", "4:8")), (
+            "ViT-L/16 linears, batch 32 (T=6304), FP16, N:M in {1:4,2:4,2:8,4:8} with one pattern per "
+            "128-channel tile, activation feature-major, gather SpMM")
     else:
         raise SystemExit(f"unknown config {name}")
+    if _ONLY:  # profiling one kernel shape of the config
+        ls = [l for l in ls if f"{l.name}/{l.nm}" in _ONLY]
+        if not ls:
+            raise SystemExit(f"--only matched no problem of config {name}: {_ONLY}")
+        desc = f"{desc}; only {','.join(_ONLY)}"
     stream = torch.cuda.current_stream()
     probs = []
     int8out = name == "int8out"
+    gather = name in ("gather", "gatherl")
     for l in ls:
         W, X, sc = l.weight().cuda(), l.activation().cuda(), l.scale()
         sc = None if sc is None else sc.cuda()
+        if gather:
+            h = nm.nm_compress_tile(W, l.N, l.M)
+            Xt = X.t().contiguous()
+            Y = torch.empty((l.T, l.n_out), dtype=nm.out_dtype(h, sc is not None), device="cuda")
+            call = (lambda st, h=h, Xt=Xt, Y=Y, sc=sc: nm.nm_spmm_gather(h, Xt, Y=Y, scale=sc, stream=st))
+            probs.append((l, W, X, sc, h, Y, call))
+            continue
         h = nm.nm_compress(W, l.N, l.M)
         if int8out:  # per-channel bias; GELU after fc1; one int8 step = 10 output units
             bias = inputs.normal_f32((l.n_out,), 5.0, l.seed + 3).cuda()
@@ -462,7 +513,14 @@ def run_config(name: str, args) -> None:
     per = []
     for i, (l, W, X, sc, h, Y, _) in enumerate(probs):
         us = statistics.median(evs[r][i][0].elapsed_time(evs[r][i][1]) * 1e3 for r in range(reps))
-        rp = roofline_point(l, us, pk, 1 if int8out else None, int8out)
+        rp = roofline_point(l, us, pk, 1 if int8out else None, int8out, gather)
+        if gather:  # the same weight with per-row patterns through nm_spmm (token-major X), same timing
+            he = nm.nm_compress(W, l.N, l.M)
+            Ye = torch.empty_like(Y)
+            rp["per_row_patterns_us"] = round(_graph_us(lambda st: nm.nm_spmm(he, X, Y=Ye, scale=sc, stream=st),
+                                                        stream), 2)
+            rp["gather_graph_us"] = round(_graph_us(lambda st: probs[i][6](st), stream), 2)
+            he.destroy()
         # same-shape cuBLAS dense GEMM through torch (context)
         if l.dtype == inputs.INT8 and l.T > 16:
             fn = (lambda X=X, W=W: torch._int_mm(X, W.t()))
@@ -509,7 +567,8 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
-    ap.add_argument("--config", default=None, choices=["single", "vitl", "swin", "mixed1", "mixed256", "int8out", "lut", "search"],
+    ap.add_argument("--config", default=None, choices=["single", "vitl", "swin", "mixed1", "mixed256", "int8out", "gather",
+                                                       "gatherl", "lut", "search"],
                     help="measure another workload (one JSON line) instead of the default ViT-B INT8 set")
     ap.add_argument("--only", action="append", default=[],
                     help="restrict to problems like vitb.fc1/2:4 (profiling a single kernel shape)")
