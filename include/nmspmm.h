@@ -221,9 +221,11 @@ nm_status nm_compress_tile(const void* W_dev, int64_t n_out, int64_t k, nm_dtype
  * nm_spmm_gather -- Y = X . Wm^T for a handle made by nm_compress_tile, with
  * the activation given feature-major: Xt_dev [k][ldx] holds X[t][kk] at
  * Xt_dev[kk * ldx + t].  Per 128-channel tile the kernel gathers the kept rows
- * of Xt (tensor-memory-access gathers of four rows per copy) into a dense
- * operand and runs dense tensor-core MMAs over K' = k * N / M only, so both
- * the MMA work and the activation bytes read per tile shrink by N / M.
+ * of Xt (16-byte asynchronous copies, eight threads per 128-byte token run)
+ * into a dense operand and runs dense tensor-core MMAs over K' = k * N / M
+ * only, so both the MMA work and the activation bytes read per tile shrink by
+ * N / M.  Environment NMSPMM_GATHER_TMA=1 gathers with four-row tensor copies
+ * instead (same results; slower on B200).
  *
  * Xt_dev    16-byte aligned; ldx >= T and ldx * sizeof(dtype) a multiple of
  *           16 bytes (else NM_ERR_INVALID).  Columns t >= T are not read.
