@@ -256,3 +256,35 @@ def test_gather_contract_errors():
     st = L.nm_spmm_gather(th.raw, Xt.data_ptr(), 64, 64, ctypes.c_void_p(Y.data_ptr() + 4), None, None)
     assert st == nm.NM_ERR_INVALID
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("N,M", [(1, 4), (2, 8), (4, 8)])
+def test_gather_extreme_values_bit_exact(N, M):
+    """Largest accumulator magnitudes through the gather: X = -128 everywhere and
+    weights at +-127 (every column mass ties, so the tie rule picks every kept k)."""
+    n_out, K, T = 256, 4096, 130
+    sign = torch.where(inputs.int8_uniform((n_out, K), 0, 1, seed=71) > 0, 127, -127).to(torch.int8)
+    sign[:8] = 127
+    X = torch.full((T, K), -128, dtype=torch.int8)
+    h = nm.nm_compress_tile(sign.cuda(), N, M)
+    Y = nm.nm_spmm_gather(h, _feature_major(X, 0))
+    _, idx, Wm = _oracle_masked(sign.numpy(), N, M)
+    ref = oracle.gemm(X.numpy(), Wm)
+    assert np.abs(ref).max() == 128 * 127 * K * N // M
+    assert (idx[:, 0] & 0xF == 0).all()  # all masses tie: the lowest positions are kept
+    assert np.array_equal(Y.cpu().numpy(), ref)
+
+
+def test_gather_long_k_and_many_channel_tiles():
+    """K = 32768 at 2:8 (K' = 8192: 64 gather k-blocks) and n_out = 20000
+    (157 channel tiles, more than the SMs), ragged in both; sampled tokens."""
+    for (T, n_out, K, N, M, seed) in ((300, 200, 32768, 2, 8, 91), (70, 20000, 256, 1, 4, 92)):
+        W = _weights("int8", n_out, K, seed=seed)
+        X = _acts("int8", T, K, seed=seed + 1)
+        s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=seed + 2)
+        h = nm.nm_compress_tile(W.cuda(), N, M)
+        Y = nm.nm_spmm_gather(h, _feature_major(X, 32), scale=s.cuda())
+        _, _, Wm = _oracle_masked(W.numpy(), N, M)
+        rows = np.unique(np.concatenate([np.arange(0, min(T, 40)), np.arange(max(0, T - 40), T)]))
+        ref = oracle.gemm(X.numpy()[rows], Wm, scale=s.numpy())
+        assert np.array_equal(Y.cpu().numpy()[rows].view(np.uint32), ref.view(np.uint32))
