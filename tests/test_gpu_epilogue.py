@@ -121,6 +121,30 @@ def test_int8_gelu_within_erf_bound(N, M, out):
         assert np.all(np.abs(got - g) <= bound), float(np.max(np.abs(got - g) - bound))
 
 
+def test_gelu_sweep_within_bound():
+    """Dense sweep of the GELU input over [-9, 9] (an FP16 handle with one-hot
+    activations makes every pre-activation a chosen value): the kernel's fp32
+    GELU against the fp64 oracle within the stated bound."""
+    n_out, K = 512, 128
+    grid = np.linspace(-9.0, 9.0, n_out * K).reshape(n_out, K)
+    W = torch.tensor(grid, dtype=torch.float32).to(torch.float16)
+    b = torch.tensor(np.linspace(0, 4e-3, n_out), dtype=torch.float32)  # off the fp16 grid
+    X = torch.eye(K, dtype=torch.float16)                               # token t picks weight column t
+    h = nm.nm_compress(W.cuda(), 4, 4)
+    Y = nm.nm_spmm_ex(h, X.cuda(), bias=b.cuda(), act="gelu", out="float32")
+    torch.cuda.synchronize()
+    acc = W.t().double().numpy()                                        # [T = K, n_out]: exact products
+    v = oracle.epilogue(acc, None, b.numpy(), "none", "float32")["pre"]
+    g = oracle.epilogue(acc, None, b.numpy(), "gelu", "float32")["pre"]
+    got = _as_f64(Y)
+    err = np.abs(got - g)
+    bound = _gelu_tol(v, g) * (1 + 2.0 ** -24) + 2.0 ** -24 * np.abs(g)
+    worst = float(np.max(err - bound))
+    print(f"gelu sweep: max |err| {err.max():.3e}, max |err|/|v| {np.max(err / np.maximum(np.abs(v), 1e-30)):.3e}, "
+          f"excess over bound {worst:.3e}")
+    assert worst <= 0.0
+
+
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("out", ["float32", "float16", "bfloat16"])
 @pytest.mark.parametrize("act", ["none", "gelu"])
