@@ -339,6 +339,32 @@ int out_elem_bytes(const nm_handle* h, const EpiReq* ep) {
   return h->dt == nm::DT_I8 ? 4 : 2;
 }
 
+// Split-K partial tiles and per-tile arrival counters of the handle, grown
+// (after a device synchronisation: earlier launches may still use the old
+// ones) when plan `p` needs more than the handle holds.
+nm_status ensure_split_workspace(nm_handle* h, const nm::Plan& p) {
+  const int tiles = h->n_ct * p.n_tt;
+  const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
+  if (need <= h->ws_bytes && tiles <= h->cnt_len) return NM_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "synchronise before growing the split-K workspace");
+  cudaFree(h->d_ws);
+  cudaFree(h->d_cnt);
+  h->d_ws = nullptr;
+  h->d_cnt = nullptr;
+  h->ws_bytes = 0;
+  h->cnt_len = 0;
+  const int cl = std::max(tiles, 256);
+  if ((e = cudaMalloc(&h->d_ws, need)) != cudaSuccess) return cuda_fail(e, "allocate split-K workspace");
+  if ((e = cudaMalloc(&h->d_cnt, (size_t)cl * sizeof(int))) != cudaSuccess)
+    return cuda_fail(e, "allocate split-K counters");
+  if ((e = cudaMemset(h->d_cnt, 0, (size_t)cl * sizeof(int))) != cudaSuccess)
+    return cuda_fail(e, "clear split-K counters");
+  h->ws_bytes = need;
+  h->cnt_len = cl;
+  return NM_OK;
+}
+
 nm_status reject_tile(const nm_handle* h) {
   if (h->tile) return fail(NM_ERR_INVALID, "the handle was made by nm_compress_tile: its product is nm_spmm_gather");
   return NM_OK;
@@ -395,27 +421,7 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   if (const char* tp = getenv("NMSPMM_TRACE_PTR")) a.trace = reinterpret_cast<long long*>(strtoull(tp, nullptr, 0));
 #endif
   if (p.splits > 1) {
-    const int tiles = h->n_ct * p.n_tt;
-    const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
-    if (need > h->ws_bytes || tiles > h->cnt_len) {
-      cudaError_t e = cudaDeviceSynchronize();
-      if (e != cudaSuccess) return cuda_fail(e, "synchronise before growing the split-K workspace");
-      cudaFree(h->d_ws);
-      cudaFree(h->d_cnt);
-      h->d_ws = nullptr;
-      h->d_cnt = nullptr;
-      h->ws_bytes = 0;
-      h->cnt_len = 0;
-      const size_t ws = std::max(need, h->ws_bytes);
-      const int cl = std::max(tiles, 256);
-      if ((e = cudaMalloc(&h->d_ws, ws)) != cudaSuccess) return cuda_fail(e, "allocate split-K workspace");
-      if ((e = cudaMalloc(&h->d_cnt, (size_t)cl * sizeof(int))) != cudaSuccess)
-        return cuda_fail(e, "allocate split-K counters");
-      if ((e = cudaMemset(h->d_cnt, 0, (size_t)cl * sizeof(int))) != cudaSuccess)
-        return cuda_fail(e, "clear split-K counters");
-      h->ws_bytes = ws;
-      h->cnt_len = cl;
-    }
+    if ((st = ensure_split_workspace(h, p)) != NM_OK) return st;
     a.ws = h->d_ws;
     a.cnt = h->d_cnt;
   }
@@ -704,26 +710,7 @@ nm_status nm_spmm_gather(const nm_handle* hc, const void* Xt, int64_t ldx, int64
   // four-row tensor gathers, whose per-copy cost caps them near 1.3 TB/s.
   a.gather_tma = env_int("NMSPMM_GATHER_TMA", 0) ? 1 : 0;
   if (p.splits > 1) {
-    const int tiles = h->n_ct * p.n_tt;
-    const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
-    if (need > h->ws_bytes || tiles > h->cnt_len) {
-      cudaError_t e = cudaDeviceSynchronize();
-      if (e != cudaSuccess) return cuda_fail(e, "synchronise before growing the split-K workspace");
-      cudaFree(h->d_ws);
-      cudaFree(h->d_cnt);
-      h->d_ws = nullptr;
-      h->d_cnt = nullptr;
-      h->ws_bytes = 0;
-      h->cnt_len = 0;
-      const int cl = std::max(tiles, 256);
-      if ((e = cudaMalloc(&h->d_ws, need)) != cudaSuccess) return cuda_fail(e, "allocate split-K workspace");
-      if ((e = cudaMalloc(&h->d_cnt, (size_t)cl * sizeof(int))) != cudaSuccess)
-        return cuda_fail(e, "allocate split-K counters");
-      if ((e = cudaMemset(h->d_cnt, 0, (size_t)cl * sizeof(int))) != cudaSuccess)
-        return cuda_fail(e, "clear split-K counters");
-      h->ws_bytes = need;
-      h->cnt_len = cl;
-    }
+    if ((st = ensure_split_workspace(h, p)) != NM_OK) return st;
     a.ws = h->d_ws;
     a.cnt = h->d_cnt;
   }
