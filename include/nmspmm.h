@@ -239,6 +239,16 @@ nm_status nm_spmm_gather(const nm_handle* h, const void* Xt_dev, int64_t ldx, in
                          const float* scale_dev, void* stream);
 
 /*
+ * nm_spmm_gather_ex -- nm_spmm_gather with the fused output stage of
+ * nm_spmm_ex (nm_epilogue above): Y = out(act((X . Wm^T) * scale + bias)), the same
+ * definition, element types, rounding and argument checks as nm_spmm_ex; the
+ * activation arguments (Xt_dev, ldx, T) and their checks are those of
+ * nm_spmm_gather.  ep == NULL is nm_spmm_gather without a scale.
+ */
+nm_status nm_spmm_gather_ex(const nm_handle* h, const void* Xt_dev, int64_t ldx, int64_t T, void* Y_dev,
+                            const nm_epilogue* ep, void* stream);
+
+/*
  * nm_decompress -- write the masked dense weight Wm [n_out][k] (dtype of the
  * handle) decoded from the packed operand image the SpMM kernel reads, so the
  * image can be checked against the top-N rule.  W_dev_out 16-byte aligned.

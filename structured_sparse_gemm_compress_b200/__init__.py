@@ -25,7 +25,7 @@ _ELEM = {NM_INT8: torch.int8, NM_FP16: torch.float16, NM_BF16: torch.bfloat16}
 
 # Every symbol include/nmspmm.h declares.
 EXPORTS = ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_ex", "nm_spmm_gather",
-           "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
+           "nm_spmm_gather_ex", "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
            "nm_device_status", "nm_destroy", "nm_last_error", "nm_version", "nm_test_spmm_skip_stage")
 
 
@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         L.nm_compress.argtypes = [vp, i64, i64, i32, i32, i32, vp, ctypes.POINTER(vp)]
         L.nm_compress_tile.argtypes = [vp, i64, i64, i32, i32, i32, vp, ctypes.POINTER(vp)]
         L.nm_spmm_gather.argtypes = [vp, vp, i64, i64, vp, vp, vp]
+        L.nm_spmm_gather_ex.argtypes = [vp, vp, i64, i64, vp, ctypes.POINTER(NMEpilogue), vp]
         L.nm_recompress.argtypes = [vp, vp, vp]
         L.nm_spmm.argtypes = [vp, vp, i64, vp, vp, vp]
         L.nm_spmm_noalloc.argtypes = [vp, vp, i64, vp, vp, vp]
@@ -65,7 +66,8 @@ def lib() -> ctypes.CDLL:
         L.nm_destroy.restype = None
         L.nm_last_error.restype = ctypes.c_char_p
         L.nm_version.restype = ctypes.c_char_p
-        for name in ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_gather", "nm_spmm_noalloc",
+        for name in ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_gather",
+                     "nm_spmm_gather_ex", "nm_spmm_noalloc",
                      "nm_test_spmm_skip_stage", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
                      "nm_device_status"):
             getattr(L, name).restype = i32
@@ -241,6 +243,30 @@ def nm_spmm_ex(h: NMHandle, X: torch.Tensor, Y: torch.Tensor | None = None, scal
         raise ValueError(f"Y must be a contiguous [{T}, {h.n_out}] {want} tensor")
     ep = NMEpilogue(OUT_TYPES[out], ACTS[act], _ptr(scale), _ptr(bias), float(out_scale))
     _check(lib().nm_spmm_ex(h.raw, _ptr(X), T, _ptr(Y), ctypes.byref(ep), _stream(stream)))
+    return Y
+
+
+def nm_spmm_gather_ex(h: NMHandle, Xt: torch.Tensor, T: int | None = None, Y: torch.Tensor | None = None,
+                      scale: torch.Tensor | None = None, bias: torch.Tensor | None = None, act: str = "none",
+                      out: str = "default", out_scale: float = 1.0, stream=None) -> torch.Tensor:
+    """``nm_spmm_gather`` (feature-major ``Xt`` [k, ldx], tile-shared handle)
+    with the fused output stage of ``nm_spmm_ex``."""
+    if Xt.dtype != h.dtype or not Xt.is_cuda or Xt.dim() != 2 or Xt.shape[0] != h.k or Xt.stride(1) != 1:
+        raise ValueError("Xt must be a CUDA [k, T] tensor of the handle's dtype with contiguous rows")
+    if out not in OUT_TYPES or act not in ACTS:
+        raise ValueError(f"out must be one of {tuple(OUT_TYPES)}, act one of {tuple(ACTS)}")
+    for name, v in (("scale", scale), ("bias", bias)):
+        if v is not None and (v.dtype != torch.float32 or v.numel() != h.n_out or not v.is_cuda):
+            raise ValueError(f"{name} must be a CUDA float32 tensor of n_out elements")
+    T = Xt.shape[1] if T is None else int(T)
+    want = _OUT_TORCH[resolve_out(h, out, scale, bias, act)]
+    if Y is None:
+        Y = torch.empty((T, h.n_out), dtype=want, device=Xt.device)
+    elif Y.dtype != want or tuple(Y.shape) != (T, h.n_out) or not Y.is_contiguous():
+        raise ValueError(f"Y must be a contiguous [{T}, {h.n_out}] {want} tensor")
+    ep = NMEpilogue(OUT_TYPES[out], ACTS[act], _ptr(scale), _ptr(bias), float(out_scale))
+    ldx = Xt.stride(0) if Xt.shape[0] > 1 else Xt.shape[1]
+    _check(lib().nm_spmm_gather_ex(h.raw, _ptr(Xt), ldx, T, _ptr(Y), ctypes.byref(ep), _stream(stream)))
     return Y
 
 

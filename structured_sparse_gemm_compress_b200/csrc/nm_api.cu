@@ -365,6 +365,36 @@ nm_status ensure_split_workspace(nm_handle* h, const nm::Plan& p) {
   return NM_OK;
 }
 
+// Validates the output stage `ep` for handle `h`.  *fixed: the fixed stages
+// of nm_spmm compute exactly these values (r is then unused); otherwise r is
+// the runtime stage to run.
+nm_status resolve_epilogue(const nm_handle* h, const nm_epilogue* ep, bool* fixed, EpiReq* r) {
+  if ((int)ep->out < 0 || (int)ep->out > 5) return fail(NM_ERR_INVALID, "unknown output type %d", (int)ep->out);
+  if ((int)ep->act < 0 || (int)ep->act > 1) return fail(NM_ERR_INVALID, "unknown activation %d", (int)ep->act);
+  if ((ep->scale && !aligned(ep->scale, 4)) || (ep->bias && !aligned(ep->bias, 4)))
+    return fail(NM_ERR_INVALID, "scale and bias must be 4-byte aligned");
+  const bool plain = !ep->scale && !ep->bias && ep->act == NM_ACT_NONE;
+  const bool int_in = h->dt == nm::DT_I8;
+  nm_out_type out = ep->out;
+  if (out == NM_OUT_DEFAULT)
+    out = int_in ? (plain ? NM_OUT_INT32 : NM_OUT_FP32) : (h->dt == nm::DT_F16 ? NM_OUT_FP16 : NM_OUT_BF16);
+  if (!int_in && (out == NM_OUT_INT32 || out == NM_OUT_INT8))
+    return fail(NM_ERR_UNSUPPORTED, "integer outputs need an INT8 handle");
+  if (out == NM_OUT_INT32 && !plain)
+    return fail(NM_ERR_INVALID, "NM_OUT_INT32 is the raw accumulator: no scale, bias or activation");
+  if (out == NM_OUT_INT8 && !(std::isfinite(ep->out_scale) && ep->out_scale > 0.0f))
+    return fail(NM_ERR_INVALID, "out_scale must be finite and positive for NM_OUT_INT8");
+  *fixed = ep->act == NM_ACT_NONE && !ep->bias &&
+           ((int_in && out == NM_OUT_INT32) || (int_in && out == NM_OUT_FP32 && ep->scale) ||
+            (h->dt == nm::DT_F16 && out == NM_OUT_FP16) || (h->dt == nm::DT_BF16 && out == NM_OUT_BF16));
+  r->out_ty = out == NM_OUT_FP32 ? nm::OUT_F32 : out == NM_OUT_FP16 ? nm::OUT_F16 : out == NM_OUT_BF16 ? nm::OUT_BF16
+                                                                                                       : nm::OUT_I8;
+  r->bias = ep->bias;
+  r->act = ep->act == NM_ACT_GELU ? nm::ACT_GELU : nm::ACT_NONE;
+  r->out_scale = ep->out_scale;
+  return NM_OK;
+}
+
 nm_status reject_tile(const nm_handle* h) {
   if (h->tile) return fail(NM_ERR_INVALID, "the handle was made by nm_compress_tile: its product is nm_spmm_gather");
   return NM_OK;
@@ -469,6 +499,10 @@ nm_status noalloc_scratch(int dev, void** out) {
   return NM_OK;
 }
 
+// nm_spmm_gather / nm_spmm_gather_ex (defined after the exported calls that use it).
+nm_status gather_impl(const nm_handle* hc, const void* Xt, int64_t ldx, int64_t T, void* Y, const float* scale,
+                      void* stream, const EpiReq* ep);
+
 }  // namespace
 
 extern "C" {
@@ -559,33 +593,10 @@ nm_status nm_spmm_ex(const nm_handle* h, const void* X_dev, int64_t T, void* Y_d
   if (!ep) return spmm_impl(h, X_dev, T, Y_dev, nullptr, stream, -1, 1000000000ull);
   nm_status st = check_handle(h);
   if (st != NM_OK) return st;
-  if ((int)ep->out < 0 || (int)ep->out > 5) return fail(NM_ERR_INVALID, "unknown output type %d", (int)ep->out);
-  if ((int)ep->act < 0 || (int)ep->act > 1) return fail(NM_ERR_INVALID, "unknown activation %d", (int)ep->act);
-  if ((ep->scale && !aligned(ep->scale, 4)) || (ep->bias && !aligned(ep->bias, 4)))
-    return fail(NM_ERR_INVALID, "scale and bias must be 4-byte aligned");
-  const bool plain = !ep->scale && !ep->bias && ep->act == NM_ACT_NONE;
-  const bool int_in = h->dt == nm::DT_I8;
-  nm_out_type out = ep->out;
-  if (out == NM_OUT_DEFAULT)
-    out = int_in ? (plain ? NM_OUT_INT32 : NM_OUT_FP32) : (h->dt == nm::DT_F16 ? NM_OUT_FP16 : NM_OUT_BF16);
-  if (!int_in && (out == NM_OUT_INT32 || out == NM_OUT_INT8))
-    return fail(NM_ERR_UNSUPPORTED, "integer outputs need an INT8 handle");
-  if (out == NM_OUT_INT32 && !plain)
-    return fail(NM_ERR_INVALID, "NM_OUT_INT32 is the raw accumulator: no scale, bias or activation");
-  if (out == NM_OUT_INT8 && !(std::isfinite(ep->out_scale) && ep->out_scale > 0.0f))
-    return fail(NM_ERR_INVALID, "out_scale must be finite and positive for NM_OUT_INT8");
-  // The fixed stages of nm_spmm compute the same values; use them where they apply.
-  const bool fixed = ep->act == NM_ACT_NONE && !ep->bias &&
-                     ((int_in && out == NM_OUT_INT32) || (int_in && out == NM_OUT_FP32 && ep->scale) ||
-                      (h->dt == nm::DT_F16 && out == NM_OUT_FP16) || (h->dt == nm::DT_BF16 && out == NM_OUT_BF16));
-  if (fixed) return spmm_impl(h, X_dev, T, Y_dev, ep->scale, stream, -1, 1000000000ull);
+  bool fixed = false;
   EpiReq r;
-  r.out_ty = out == NM_OUT_FP32 ? nm::OUT_F32 : out == NM_OUT_FP16 ? nm::OUT_F16 : out == NM_OUT_BF16 ? nm::OUT_BF16
-                                                                                                      : nm::OUT_I8;
-  r.bias = ep->bias;
-  r.act = ep->act == NM_ACT_GELU ? nm::ACT_GELU : nm::ACT_NONE;
-  r.out_scale = ep->out_scale;
-  return spmm_impl(h, X_dev, T, Y_dev, ep->scale, stream, -1, 1000000000ull, &r);
+  if ((st = resolve_epilogue(h, ep, &fixed, &r)) != NM_OK) return st;
+  return spmm_impl(h, X_dev, T, Y_dev, ep->scale, stream, -1, 1000000000ull, fixed ? nullptr : &r);
 }
 
 nm_status nm_test_spmm_skip_stage(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
@@ -666,6 +677,28 @@ nm_status nm_spmm_gather(const nm_handle* hc, const void* Xt, int64_t ldx, int64
   g_err.clear();
   nm_status st = check_handle(hc);
   if (st != NM_OK) return st;
+  return gather_impl(hc, Xt, ldx, T, Y, scale, stream, nullptr);
+}
+
+nm_status nm_spmm_gather_ex(const nm_handle* h, const void* Xt, int64_t ldx, int64_t T, void* Y,
+                            const nm_epilogue* ep, void* stream) {
+  g_err.clear();
+  nm_status st = check_handle(h);
+  if (st != NM_OK) return st;
+  if (!ep) return gather_impl(h, Xt, ldx, T, Y, nullptr, stream, nullptr);
+  bool fixed = false;
+  EpiReq r;
+  if ((st = resolve_epilogue(h, ep, &fixed, &r)) != NM_OK) return st;
+  return gather_impl(h, Xt, ldx, T, Y, ep->scale, stream, fixed ? nullptr : &r);
+}
+
+}  // extern "C"
+
+namespace {
+
+nm_status gather_impl(const nm_handle* hc, const void* Xt, int64_t ldx, int64_t T, void* Y, const float* scale,
+                      void* stream, const EpiReq* ep) {
+  nm_status st = NM_OK;
   if (!hc->tile) return fail(NM_ERR_INVALID, "nm_spmm_gather needs a handle made by nm_compress_tile");
   nm_handle* h = const_cast<nm_handle*>(hc);  // only caches (tensor map, workspace) change
   if (T < 0) return fail(NM_ERR_INVALID, "T must be >= 0 (got %lld)", (long long)T);
@@ -678,7 +711,7 @@ nm_status nm_spmm_gather(const nm_handle* hc, const void* Xt, int64_t ldx, int64
     return fail(NM_ERR_INVALID, "ldx * sizeof(dtype) must be a multiple of 16 bytes (ldx=%lld)", (long long)ldx);
   if (!aligned(Xt, 16) || !aligned(Y, 16)) return fail(NM_ERR_INVALID, "Xt and Y must be 16-byte aligned");
   if (scale && !aligned(scale, 4)) return fail(NM_ERR_INVALID, "scale must be 4-byte aligned");
-  const size_t ybytes = (size_t)T * h->n_out * out_elem_bytes(h, nullptr);
+  const size_t ybytes = (size_t)T * h->n_out * out_elem_bytes(h, ep);
   const size_t xbytes = ((size_t)(h->k - 1) * ldx + T) * es;
   const uintptr_t xs = (uintptr_t)Xt, ys = (uintptr_t)Y;
   if (xs < ys + ybytes && ys < xs + xbytes) return fail(NM_ERR_INVALID, "Y overlaps Xt");
@@ -709,6 +742,10 @@ nm_status nm_spmm_gather(const nm_handle* hc, const void* Xt, int64_t ldx, int64
   // Gather warps (load/store path) by default: measured faster on B200 than
   // four-row tensor gathers, whose per-copy cost caps them near 1.3 TB/s.
   a.gather_tma = env_int("NMSPMM_GATHER_TMA", 0) ? 1 : 0;
+  a.out_ty = ep ? ep->out_ty : -1;
+  a.bias = ep ? ep->bias : nullptr;
+  a.act = ep ? ep->act : nm::ACT_NONE;
+  a.out_scale = ep ? ep->out_scale : 1.0f;
   if (p.splits > 1) {
     if ((st = ensure_split_workspace(h, p)) != NM_OK) return st;
     a.ws = h->d_ws;
@@ -717,6 +754,10 @@ nm_status nm_spmm_gather(const nm_handle* hc, const void* Xt, int64_t ldx, int64
   cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch SpMM kernel");
 }
+
+}  // namespace
+
+extern "C" {
 
 nm_status nm_decompress(const nm_handle* h, void* W_dev_out, void* stream) {
   g_err.clear();

@@ -54,9 +54,13 @@ constexpr int out_bytes(int out) { return ((out & 3) == OUT_I32 || (out & 3) == 
 // Epilogue warps and CTA size of a kernel with output code OUT.
 constexpr int epi_warps(int out) { return 4 * epw_for((out & kOutEpi) != 0); }
 constexpr int cta_threads(int out) { return 64 + 32 * epi_warps(out); }
-// Gather image: warps that gather the kept activation rows (after the epilogue warps).
-constexpr int kGatherWarps = 8;
-constexpr int kernel_threads(int img, int out) { return cta_threads(out) + (img == IMG_GATHER ? 32 * kGatherWarps : 0); }
+// Gather image: warps that gather the kept activation rows (after the epilogue
+// warps): 8, or 4 beside the runtime output stage's 16 epilogue warps (which
+// keeps every thread within 88 registers).
+__host__ __device__ constexpr int gather_warps(int out) { return (out & kOutEpi) ? 4 : 8; }
+constexpr int kernel_threads(int img, int out) {
+  return cta_threads(out) + (img == IMG_GATHER ? 32 * gather_warps(out) : 0);
+}
 
 // Kernel configuration.  XKB = 0: streaming mode, every stage carries a packed
 // weight chunk and the matching X boxes.  XKB > 0: X-stationary mode, the
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
 
   if (threadIdx.x == 0) {
     // gather image with gather warps: the producer's arrive plus one per gather warp
-    const uint32_t full_count = (C::GA && !a.gather_tma) ? 1u + kGatherWarps : 1u;
+    const uint32_t full_count = (C::GA && !a.gather_tma) ? 1u + gather_warps(OUT) : 1u;
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full_bar[i], full_count);
       mbar_init(&empty_bar[i], 1);
@@ -631,7 +635,7 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
     if constexpr (C::GA) {
       if (!a.gather_tma) {
         constexpr int ES = elem_bytes(DT);
-        constexpr int RSTEP = 32 * kGatherWarps / 8;  // kept rows per pass
+        constexpr int RSTEP = 32 * gather_warps(OUT) / 8;  // kept rows per pass
         constexpr int PASSES = C::KB / RSTEP;
         constexpr int TOK = 128 / ES;                 // tokens per 128-byte run
         constexpr int LAG = 2;
@@ -1272,11 +1276,11 @@ static cudaError_t launch_bn(const CUtensorMap* tmX, const CUtensorMap* tmY, con
   }
 }
 
-// Gather image: streaming kernel only, fixed output stages with direct stores.
+// Gather image: streaming kernel only, direct-store output stages (fixed or runtime).
 template <int DT, int OUT>
 static cudaError_t launch_gather(const CUtensorMap* tmX, const CUtensorMap* tmY, const CUtensorMap* tmW,
                                  const Plan& p, const SpmmArgs& a, cudaStream_t s) {
-  if constexpr (DT != DT_BF16 && (OUT & kOutEpi) == 0 && (OUT & kOutDirect) != 0) {
+  if constexpr (DT != DT_BF16 && (OUT & kOutDirect) != 0) {
     if (p.pair || p.xkb > 0) return cudaErrorInvalidValue;
     switch (p.bn) {
       case 128: return launch_t<DT, IMG_GATHER, 128, OUT, 0>(tmX, tmY, tmW, p, a, s);

@@ -288,3 +288,74 @@ def test_gather_long_k_and_many_channel_tiles():
         rows = np.unique(np.concatenate([np.arange(0, min(T, 40)), np.arange(max(0, T - 40), T)]))
         ref = oracle.gemm(X.numpy()[rows], Wm, scale=s.numpy())
         assert np.array_equal(Y.cpu().numpy()[rows].view(np.uint32), ref.view(np.uint32))
+
+
+# --------------------------------------------------------------------------- gather + fused output stage
+
+
+def _epi_problem(N, M, T=300, n_out=200, K=784):
+    W = _weights("int8", n_out, K, seed=401)
+    X = _acts("int8", T, K, seed=402)
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=403)
+    b = inputs.normal_f32((n_out,), 20.0, seed=404)
+    _, _, Wm = _oracle_masked(W.numpy(), N, M)
+    return W, X, s, b, oracle.gemm(X.numpy(), Wm)
+
+
+def _as_bits(Y: torch.Tensor) -> np.ndarray:
+    Y = Y.cpu()
+    if Y.dtype == torch.bfloat16:
+        return Y.view(torch.int16).numpy().view(np.uint16)
+    return Y.numpy()
+
+
+@pytest.mark.parametrize("N,M", [(2, 8), (4, 8), (1, 4)])
+@pytest.mark.parametrize("out", ["float32", "float16", "bfloat16", "int8"])
+def test_gather_ex_outputs_bit_exact(N, M, out):
+    """INT8 handle, scale + bias, no activation: every output type bit-exact."""
+    W, X, s, b, acc = _epi_problem(N, M)
+    os_ = 0.25
+    h = nm.nm_compress_tile(W.cuda(), N, M)
+    Y = nm.nm_spmm_gather_ex(h, _feature_major(X, 16), scale=s.cuda(), bias=b.cuda(), out=out, out_scale=os_)
+    ref = oracle.epilogue(acc, s.numpy(), b.numpy(), "none", out, os_)["exact"]
+    assert np.array_equal(_as_bits(Y), ref)
+
+
+@pytest.mark.parametrize("N,M", [(2, 8), (4, 8)])
+def test_gather_ex_int8_gelu_within_bound(N, M):
+    """GELU then int8: a code may differ by one only where the oracle's
+    unrounded value is within the GELU bound of a half-integer."""
+    W, X, s, b, acc = _epi_problem(N, M)
+    os_ = 2.0
+    h = nm.nm_compress_tile(W.cuda(), N, M)
+    Y = nm.nm_spmm_gather_ex(h, _feature_major(X, 0), scale=s.cuda(), bias=b.cuda(), act="gelu", out="int8",
+                             out_scale=os_)
+    v = oracle.epilogue(acc, s.numpy(), b.numpy(), "none", "float32")["pre"]
+    r = oracle.epilogue(acc, s.numpy(), b.numpy(), "gelu", "int8", os_)
+    g = r["pre"]
+    tol = 4e-7 * np.abs(v) + 2e-6 * np.abs(g) + 1e-30
+    q = Y.cpu().numpy().astype(np.int64)
+    diff = np.abs(q - r["q"].astype(np.int64))
+    assert diff.max() <= 1
+    slack = os_ * tol + 2.0 ** -23 * np.abs(r["q_pre"]) + 1e-6
+    near = np.abs(np.abs(r["q_pre"] - np.floor(r["q_pre"])) - 0.5) <= slack
+    assert np.all(near[diff == 1])
+    assert (diff == 0).mean() > 0.999
+
+
+def test_gather_ex_fp16_handle_and_fixed_routing():
+    W = _weights("fp16", 256, 512, seed=411)
+    X = _acts("fp16", 150, 512, seed=412)
+    b = inputs.normal_f32((256,), 0.5, seed=413)
+    h = nm.nm_compress_tile(W.cuda(), 2, 8)
+    Xt = _feature_major(X, 8)
+    _, _, Wm = _oracle_masked(_np(W), 2, 8)
+    acc = oracle.gemm(_np(X), Wm)
+    Y = nm.nm_spmm_gather_ex(h, Xt, bias=b.cuda(), out="float32")
+    ref = oracle.epilogue(acc, None, b.numpy(), "none", "float32")["pre"]
+    err = np.abs(Y.double().cpu().numpy() - ref)
+    assert err.max() <= 2e-3 * np.abs(ref).max()
+    # no output stage requested: the fixed stage, identical to nm_spmm_gather
+    assert torch.equal(nm.nm_spmm_gather_ex(h, Xt), nm.nm_spmm_gather(h, Xt))
+    with pytest.raises(nm.NMError):
+        nm.nm_spmm_gather_ex(h, Xt, out="int8")   # integer outputs need an INT8 handle
