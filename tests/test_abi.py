@@ -78,3 +78,36 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(nm, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="missing"):
         nm.lib()
+
+
+def test_header_compiles_as_c_and_cpp(tmp_path):
+    """include/nmspmm.h is a plain C header: a C99 and a C++11 translation unit
+    that take the address of every declared entry point compile cleanly."""
+    refs = "\n".join(f"    (void)&{f};" for f in declared_functions())
+    src = f'#include "nmspmm.h"\nint main(void) {{\n{refs}\n    return 0;\n}}\n'
+    for cc, std, ext in (("gcc", "-std=c99", "c"), ("g++", "-std=c++11", "cpp")):
+        path = tmp_path / f"use_header.{ext}"
+        path.write_text(src)
+        subprocess.check_call([cc, std, "-Wall", "-Wextra", "-Werror", "-pedantic", "-I",
+                               os.path.dirname(HEADER), "-c", str(path), "-o", str(tmp_path / f"use_{ext}.o")])
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, 4, 8, nm.NM_INT8, 2, 4), nm.NM_ERR_INVALID),          # null W
+    ((16, 4, 8, nm.NM_BF16, 2, 4), nm.NM_ERR_UNSUPPORTED),        # bfloat16 column sums are not exact
+    ((16, 4, 8, nm.NM_INT8, 3, 4), nm.NM_ERR_UNSUPPORTED),        # 3:4
+    ((16, 4, 10, nm.NM_INT8, 2, 4), nm.NM_ERR_INVALID),           # k % M != 0
+    ((17, 4, 8, nm.NM_FP16, 2, 4), nm.NM_ERR_INVALID),            # misaligned fp16 W
+])
+def test_compress_tile_rejects_before_touching_the_device(args, status):
+    out = ctypes.c_void_p(123)
+    st = nm.lib().nm_compress_tile(*args, None, ctypes.byref(out))
+    assert st == status
+    assert out.value is None
+    assert nm.nm_last_error() != ""
+
+
+def test_gather_null_handle_paths():
+    L = nm.lib()
+    assert L.nm_spmm_gather(None, None, 0, 0, None, None, None) == nm.NM_ERR_INVALID
+    assert L.nm_spmm_gather_ex(None, None, 0, 0, None, None, None) == nm.NM_ERR_INVALID
