@@ -37,6 +37,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "nm_oracle.c")
 _LIB = os.path.join(_HERE, "libnm_oracle.so")
+# Test hook: a prebuilt oracle library to load instead (the mutation tests load
+# deliberately broken builds of nm_oracle.c through it); never rebuilt here.
+_LIB_OVERRIDE = os.environ.get("NM_ORACLE_LIB")
 
 DTYPES = {"int8": 0, "fp16": 1, "bf16": 2}
 _lib = None
@@ -44,6 +47,8 @@ _lib = None
 
 def build(force: bool = False) -> str:
     """Compile ``nm_oracle.c`` into ``libnm_oracle.so`` next to it."""
+    if _LIB_OVERRIDE:
+        return _LIB_OVERRIDE
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".{os.getpid()}.tmp"
         subprocess.check_call(
