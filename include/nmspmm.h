@@ -233,7 +233,11 @@ nm_status nm_compress_tile(const void* W_dev, int64_t n_out, int64_t k, nm_dtype
  *           rounding exactly as nm_spmm (INT8: int32, or float32 with scale;
  *           FP16: fp16 from the fp32 accumulator).
  * scale_dev float32 [n_out] or NULL.
- * T         >= 0; T == 0 is a no-op.  Never synchronises.
+ * T         >= 0; T == 0 is a no-op.
+ * The default plan never splits k, so the call allocates nothing and never
+ * synchronises; a split-K plan forced through NMSPMM_FORCE_SPLITK uses the
+ * handle's workspace under the rules of nm_spmm (the first such call
+ * allocates it, after a device synchronisation).
  */
 nm_status nm_spmm_gather(const nm_handle* h, const void* Xt_dev, int64_t ldx, int64_t T, void* Y_dev,
                          const float* scale_dev, void* stream);
