@@ -28,6 +28,19 @@ from dataclasses import dataclass
 import numpy as np
 
 PATTERNS = {"dense": (4, 4), "4:8": (4, 8), "2:4": (2, 4), "2:8": (2, 8), "1:4": (1, 4)}
+# One pattern per 128 output channels (nm_compress_tile), run through the
+# activation gather (nm_spmm_gather, activation given feature-major): the
+# kernel side of the search-kernel co-design offers these as further choices.
+TILE_PATTERNS = {"t4:8": (4, 8), "t2:8": (2, 8), "t1:4": (1, 4)}
+
+
+def pattern_nm(pattern: str) -> tuple[int, int, bool]:
+    """(N, M, tile-shared) of a pattern name from PATTERNS or TILE_PATTERNS."""
+    if pattern in PATTERNS:
+        return (*PATTERNS[pattern], False)
+    if pattern in TILE_PATTERNS:
+        return (*TILE_PATTERNS[pattern], True)
+    raise KeyError(f"unknown pattern {pattern!r}")
 
 
 @dataclass(frozen=True)
@@ -163,28 +176,43 @@ class _Workspace:
             self.X[(T, K)] = inputs.int8_uniform((T, K), -128, 127, self.seed + T + K).cuda()
         return self.X[(T, K)]
 
+    def act_t(self, T, K):
+        """The same activation, feature-major [K, T] (the gather's layout)."""
+        if ("t", T, K) not in self.X:
+            self.X[("t", T, K)] = self.act(T, K).t().contiguous()
+        return self.X[("t", T, K)]
+
+
+def _handle_and_call(W, s, ws: "_Workspace", pattern: str, T: int, K: int, Y):
+    """Compress W for `pattern` and return (handle, launch(stream)) of one SpMM."""
+    import structured_sparse_gemm_compress_b200 as nm
+    N, M, tile = pattern_nm(pattern)
+    if tile:
+        h = nm.nm_compress_tile(W, N, M)
+        Xt = ws.act_t(T, K)
+        return h, (lambda st: nm.nm_spmm_gather(h, Xt, Y=Y, scale=s, stream=st))
+    h = nm.nm_compress(W, N, M)
+    X = ws.act(T, K)
+    return h, (lambda st: nm.nm_spmm(h, X, Y=Y, scale=s, stream=st))
+
 
 def profile(shapes: list[tuple[int, int]], patterns: list[str], Ts: list[int], reps: int = 20,
             ws: _Workspace | None = None) -> LatencyLUT:
-    """Profile ``nm_spmm`` (INT8, per-channel scale, fp32 output) for every
-    (K, n_out) in ``shapes``, pattern and token count on the current GPU."""
+    """Profile one SpMM launch (INT8, per-channel scale, fp32 output) for every
+    (K, n_out) in ``shapes``, pattern and token count on the current GPU:
+    ``nm_spmm`` for PATTERNS, ``nm_spmm_gather`` for TILE_PATTERNS."""
     import torch
-
-    import structured_sparse_gemm_compress_b200 as nm
 
     ws = ws or _Workspace()
     table = {}
     for K, n_out in shapes:
         W, s = ws.weight(K, n_out)
         for p in patterns:
-            N, M = PATTERNS[p]
-            h = nm.nm_compress(W, N, M)
             for T in Ts:
-                X = ws.act(T, K)
                 Y = torch.empty((T, n_out), dtype=torch.float32, device="cuda")
-                table[(K, n_out, p, T)] = _graph_time_us(
-                    lambda st, h=h, X=X, Y=Y: nm.nm_spmm(h, X, Y=Y, scale=s, stream=st), reps)
-            h.destroy()
+                h, call = _handle_and_call(W, s, ws, p, T, K, Y)
+                table[(K, n_out, p, T)] = _graph_time_us(call, reps)
+                h.destroy()
     meta = {"device": torch.cuda.get_device_name(), "reps": reps, "dtype": "int8", "output": "fp32 scaled"}
     return LatencyLUT(table, meta)
 
@@ -195,21 +223,20 @@ def measure_sequence(layers: list[LayerSpec], assignment: list[str], T: int, rep
     in one stream (one CUDA graph of ``reps`` passes, events around it)."""
     import torch
 
-    import structured_sparse_gemm_compress_b200 as nm
-
     ws = ws or _Workspace()
-    handles, Ys = [], []
+    handles, calls = [], []
     for l, p in zip(layers, assignment):
         W, s = ws.weight(l.K, l.n_out)
-        N, M = PATTERNS[p]
-        handles.append((nm.nm_compress(W, N, M), ws.act(T, l.K), s))
-        Ys.append(torch.empty((T, l.n_out), dtype=torch.float32, device="cuda"))
+        Y = torch.empty((T, l.n_out), dtype=torch.float32, device="cuda")
+        h, call = _handle_and_call(W, s, ws, p, T, l.K, Y)
+        handles.append((h, Y))
+        calls.append(call)
 
     def one_pass(st):
-        for (h, X, s), Y in zip(handles, Ys):
-            nm.nm_spmm(h, X, Y=Y, scale=s, stream=st)
+        for call in calls:
+            call(st)
 
     us = _graph_time_us(one_pass, reps)
-    for h, _, _ in handles:
+    for h, _ in handles:
         h.destroy()
     return us

@@ -160,13 +160,14 @@ def solve_exact(prob: Problem, resolution_us: float = 0.05) -> np.ndarray | None
     return a
 
 
-def kept_mass(W, N: int, M: int) -> float:
+def kept_mass(W, N: int, M: int, tile: bool = False) -> float:
     """Sum of |w| over the weights the library's compressor keeps (GPU): the
-    values exported from an ``nm_compress`` handle."""
+    values exported from an ``nm_compress`` handle (``nm_compress_tile`` when
+    ``tile``: one pattern per 128 output channels)."""
     import torch
 
     import structured_sparse_gemm_compress_b200 as nm
-    h = nm.nm_compress(W, N, M)
+    h = nm.nm_compress_tile(W, N, M) if tile else nm.nm_compress(W, N, M)
     values, _ = nm.nm_export(h)
     h.destroy()
     return float(values.to(torch.float64).abs().sum())

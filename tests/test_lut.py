@@ -75,3 +75,14 @@ def test_vit_b_layers_and_assignments():
     assert len(ls) == 48 and ls[2] == lut.LayerSpec("b0.fc1", 768, 3072)
     a1, a2 = lut.random_assignment(48, 5), lut.random_assignment(48, 5)
     assert a1 == a2 and set(a1) <= set(lut.PATTERNS)
+
+
+def test_pattern_names_cover_both_families():
+    assert lut.pattern_nm("2:4") == (2, 4, False)
+    assert lut.pattern_nm("dense") == (4, 4, False)
+    assert lut.pattern_nm("t2:8") == (2, 8, True)
+    assert lut.pattern_nm("t4:8") == (4, 8, True)
+    with pytest.raises(KeyError):
+        lut.pattern_nm("t3:8")
+    asg = lut.random_assignment(200, 3, tuple(lut.PATTERNS) + tuple(lut.TILE_PATTERNS))
+    assert set(asg) == set(lut.PATTERNS) | set(lut.TILE_PATTERNS)
