@@ -392,7 +392,7 @@ def run_cosearch(args) -> None:
     ws = lut._Workspace()
     L = lut.profile(shapes, pats_all, [T], reps=10, ws=ws)
     calib = []
-    for i in range(4):
+    for i in range(6):
         asg = lut.random_assignment(len(layers), 400 + i, tuple(pats_all))
         calib.append((layers, asg, T, lut.measure_sequence(layers, asg, T, reps=3, ws=ws)))
     L.calibrate(calib)
@@ -443,7 +443,8 @@ def run_cosearch(args) -> None:
                               "pattern_counts": {p: [pats_all[i] for i in fast_all].count(p) for p in pats_all
                                                  if [pats_all[i] for i in fast_all].count(p)}},
             "all_dense_predicted_us": round(dense, 1),
-            "calibration": {"a": round(L.a, 4), "b_us_per_layer": round(L.b, 3)}, "budgets": rows,
+            "calibration": {"a": round(L.a, 4), "b_us_per_layer": round(L.b, 3),
+                            "c_us_per_tile_shared_layer": round(L.c, 3)}, "budgets": rows,
             "lut_us_fc2": {p: round(L.lookup(3072, 768, p, T), 2) for p in pats_all},
             "data": "synthetic", "dtype": "int8"}
     print(json.dumps(line), flush=True)

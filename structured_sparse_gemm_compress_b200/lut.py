@@ -12,9 +12,12 @@ detail, so this module takes the plainest reading:
   nearest points outside the profiled range);
 * a configuration (one pattern per linear layer) is predicted by summing its
   layers' table entries, then calibrated against measured end-to-end sequence
-  latencies with a least-squares fit  measured ~ a * sum + b * layers  (a
-  absorbs overlap and cache effects between back-to-back launches, b a fixed
-  cost per launch).
+  latencies with a least-squares fit
+      measured ~ a * sum + b * layers + c * tile-shared layers
+  (a absorbs overlap and cache effects between back-to-back launches, b a
+  fixed cost per launch, c what a tile-shared gather launch costs in a
+  sequence beyond its isolated table entry; c is fitted only when the samples
+  contain such layers, else 0).
 
 Profiling and sequence timing run the product kernels through the package's
 binding; the table logic itself is plain host code.
@@ -32,6 +35,11 @@ PATTERNS = {"dense": (4, 4), "4:8": (4, 8), "2:4": (2, 4), "2:8": (2, 8), "1:4":
 # activation gather (nm_spmm_gather, activation given feature-major): the
 # kernel side of the search-kernel co-design offers these as further choices.
 TILE_PATTERNS = {"t4:8": (4, 8), "t2:8": (2, 8), "t1:4": (1, 4)}
+
+
+def n_tile_layers(assignment: list[str]) -> int:
+    """How many layers of an assignment use a tile-shared pattern."""
+    return sum(1 for p in assignment if p in TILE_PATTERNS)
 
 
 def pattern_nm(pattern: str) -> tuple[int, int, bool]:
@@ -69,10 +77,10 @@ class LatencyLUT:
     """Measured per-launch latency table plus the sequence calibration."""
 
     def __init__(self, table: dict[tuple[int, int, str, int], float], meta: dict | None = None,
-                 a: float = 1.0, b: float = 0.0):
+                 a: float = 1.0, b: float = 0.0, c: float = 0.0):
         self.table = dict(table)
         self.meta = dict(meta or {})
-        self.a, self.b = float(a), float(b)
+        self.a, self.b, self.c = float(a), float(b), float(c)
 
     # ---------------------------------------------------------------- lookup
     def lookup(self, K: int, n_out: int, pattern: str, T: int) -> float:
@@ -97,16 +105,23 @@ class LatencyLUT:
 
     def predict(self, layers: list[LayerSpec], assignment: list[str], T: int) -> float:
         """Calibrated end-to-end latency (us) of the layer sequence."""
-        return self.a * self.raw_sum(layers, assignment, T) + self.b * len(layers)
+        return (self.a * self.raw_sum(layers, assignment, T) + self.b * len(layers)
+                + self.c * n_tile_layers(assignment))
 
     # ---------------------------------------------------------------- calibration
     def calibrate(self, samples: list[tuple[list[LayerSpec], list[str], int, float]]) -> tuple[float, float]:
-        """Least-squares fit of measured ~ a * raw_sum + b * n_layers over
-        (layers, assignment, T, measured_us) samples; sets and returns (a, b)."""
-        A = np.array([[self.raw_sum(ls, asg, T), float(len(ls))] for ls, asg, T, _ in samples])
+        """Least-squares fit of measured ~ a * raw_sum + b * n_layers
+        (+ c * n_tile_layers when any sample has tile-shared layers) over
+        (layers, assignment, T, measured_us) samples; sets a, b, c and returns (a, b)."""
+        A = np.array([[self.raw_sum(ls, asg, T), float(len(ls)), float(n_tile_layers(asg))]
+                      for ls, asg, T, _ in samples])
         y = np.array([m for *_, m in samples])
-        if len(samples) >= 2 and np.linalg.matrix_rank(A) == 2:
+        self.c = 0.0
+        if A[:, 2].any() and len(samples) >= 3 and np.linalg.matrix_rank(A) == 3:
             sol, *_ = np.linalg.lstsq(A, y, rcond=None)
+            self.a, self.b, self.c = float(sol[0]), float(sol[1]), float(sol[2])
+        elif len(samples) >= 2 and np.linalg.matrix_rank(A[:, :2]) == 2:
+            sol, *_ = np.linalg.lstsq(A[:, :2], y, rcond=None)
             self.a, self.b = float(sol[0]), float(sol[1])
         else:  # one sample (or all with the same layer count and sum): scale only
             self.a, self.b = float(y.sum() / A[:, 0].sum()), 0.0
@@ -115,14 +130,15 @@ class LatencyLUT:
     # ---------------------------------------------------------------- persistence
     def to_json(self) -> str:
         rows = [{"K": k, "n_out": n, "pattern": p, "T": t, "us": us} for (k, n, p, t), us in sorted(self.table.items())]
-        return json.dumps({"meta": self.meta, "calibration": {"a": self.a, "b": self.b}, "entries": rows}, indent=1)
+        return json.dumps({"meta": self.meta, "calibration": {"a": self.a, "b": self.b, "c": self.c},
+                           "entries": rows}, indent=1)
 
     @staticmethod
     def from_json(text: str) -> "LatencyLUT":
         d = json.loads(text)
         table = {(r["K"], r["n_out"], r["pattern"], r["T"]): float(r["us"]) for r in d["entries"]}
         cal = d.get("calibration", {})
-        return LatencyLUT(table, d.get("meta"), cal.get("a", 1.0), cal.get("b", 0.0))
+        return LatencyLUT(table, d.get("meta"), cal.get("a", 1.0), cal.get("b", 0.0), cal.get("c", 0.0))
 
 
 # -------------------------------------------------------------------- GPU side

@@ -25,6 +25,8 @@ from dataclasses import dataclass
 
 import numpy as np
 
+from .lut import TILE_PATTERNS
+
 
 @dataclass
 class Problem:
@@ -49,11 +51,14 @@ class Problem:
 
 def make_problem(layers, lut_, T: int, keep_mass: dict, total_mass: dict, budget_us: float,
                  patterns=None) -> Problem:
-    """Per-layer latency from the calibrated LUT (a * table entry) and the
-    constant b * layers; keep_mass[(layer name, pattern)] kept |w| mass."""
+    """Per-layer latency from the calibrated LUT (a * table entry, plus c for a
+    tile-shared pattern) and the constant b * layers; keep_mass[(layer name,
+    pattern)] kept |w| mass."""
     patterns = list(patterns) if patterns else sorted({k[2] for k in lut_.table})
     L, P = len(layers), len(patterns)
-    lat = np.array([[lut_.a * lut_.lookup(l.K, l.n_out, p, T) for p in patterns] for l in layers])
+    c = getattr(lut_, "c", 0.0)
+    lat = np.array([[lut_.a * lut_.lookup(l.K, l.n_out, p, T) + (c if p in TILE_PATTERNS else 0.0)
+                     for p in patterns] for l in layers])
     keep = np.array([[keep_mass[(l.name, p)] for p in patterns] for l in layers], dtype=np.float64)
     tot = float(sum(total_mass[l.name] for l in layers))
     return Problem(patterns, lat, keep, tot, lut_.b * L, float(budget_us))

@@ -86,3 +86,24 @@ def test_pattern_names_cover_both_families():
         lut.pattern_nm("t3:8")
     asg = lut.random_assignment(200, 3, tuple(lut.PATTERNS) + tuple(lut.TILE_PATTERNS))
     assert set(asg) == set(lut.PATTERNS) | set(lut.TILE_PATTERNS)
+
+
+def test_calibration_recovers_a_per_family_term():
+    """measured = 1.1 * sum + 0.5 per layer + 3.0 per tile-shared layer is recovered
+    exactly, and predict() applies all three terms."""
+    layers = lut.vit_b_layers(blocks=1)
+    table = {(l.K, l.n_out, p, 100): 10.0 + i + 3 * j for i, l in enumerate(layers)
+             for j, p in enumerate(("2:4", "t2:8", "dense"))}
+    L = lut.LatencyLUT(table)
+    rng = np.random.default_rng(0)
+    samples = []
+    for _ in range(8):
+        asg = [rng.choice(["2:4", "t2:8", "dense"]) for _ in layers]
+        meas = 1.1 * L.raw_sum(layers, asg, 100) + 0.5 * len(layers) + 3.0 * lut.n_tile_layers(asg)
+        samples.append((layers, asg, 100, meas))
+    L.calibrate(samples)
+    assert (L.a, L.b, L.c) == pytest.approx((1.1, 0.5, 3.0))
+    asg = ["t2:8", "2:4", "t2:8", "dense"]
+    assert L.predict(layers, asg, 100) == pytest.approx(1.1 * L.raw_sum(layers, asg, 100) + 2.0 + 6.0)
+    L2 = lut.LatencyLUT.from_json(L.to_json())
+    assert L2.c == pytest.approx(3.0)
