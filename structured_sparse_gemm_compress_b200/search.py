@@ -129,10 +129,30 @@ def solve_evolutionary(prob: Problem, pop: int = 64, generations: int = 150, see
     return max(members, key=fitness)
 
 
+def polish(prob: Problem, a: np.ndarray) -> np.ndarray:
+    """Single-layer moves into the unrounded slack: while some one-layer change
+    raises the quality and keeps the exact latency within the budget, apply the
+    one that raises it most."""
+    a = a.copy()
+    L = len(a)
+    while True:
+        lat = prob.latency(a)
+        cur_keep = prob.keep[np.arange(L), a]
+        cur_lat = prob.lat[np.arange(L), a]
+        gain = prob.keep - cur_keep[:, None]                      # [L, P]
+        fits = lat - cur_lat[:, None] + prob.lat <= prob.budget + 1e-9
+        gain = np.where(fits & (gain > 1e-12), gain, -np.inf)
+        l, p = np.unravel_index(int(np.argmax(gain)), gain.shape)
+        if not np.isfinite(gain[l, p]):
+            return a
+        a[l] = p
+
+
 def solve_exact(prob: Problem, resolution_us: float = 0.05) -> np.ndarray | None:
     """Optimum of the multiple-choice knapsack by dynamic programming over
     latency in steps of ``resolution_us`` (latencies rounded up, so the result
-    is feasible; it is optimal up to that rounding)."""
+    is feasible; it is optimal up to that rounding), then ``polish`` into the
+    slack the rounding left."""
     L, P = prob.lat.shape
     cap = int(np.floor((prob.budget - prob.offset) / resolution_us + 1e-9))
     if cap < 0:
@@ -162,7 +182,7 @@ def solve_exact(prob: Problem, resolution_us: float = 0.05) -> np.ndarray | None
     for l in range(L - 1, -1, -1):
         a[l] = choice[l, c]
         c -= w[l, a[l]]
-    return a
+    return polish(prob, a)
 
 
 def kept_mass(W, N: int, M: int, tile: bool = False) -> float:

@@ -63,3 +63,29 @@ def test_unconstrained_budget_keeps_best_quality():
     prob.budget = 1e9
     for a in (search.solve_greedy(prob), search.solve_exact(prob), search.solve_evolutionary(prob, pop=16, generations=10)):
         assert prob.quality(a) == pytest.approx(prob.keep.max(axis=1).sum() / prob.total_mass)
+
+
+def test_exact_solver_recovers_what_rounding_hides():
+    """Two layers whose exact latencies fill the budget exactly: rounding every
+    latency up would make the best pair look infeasible; the polish restores it."""
+    prob = search.Problem(["fast", "good"], np.array([[1.0, 1.02], [1.0, 1.03]]),
+                          np.array([[1.0, 2.0], [1.0, 2.0]]), total_mass=4.0, offset=0.0, budget=2.03)
+    a = search.solve_exact(prob, resolution_us=0.05)
+    assert prob.feasible(a)
+    assert prob.quality(a) == pytest.approx(3.0 / 4.0)      # one layer upgraded within 2.03
+    unpolished_best = max(prob.quality(np.array(x)) for x in ([0, 0], [1, 0], [0, 1], [1, 1])
+                          if prob.latency(np.array(x)) <= 2.03 + 1e-9)
+    assert prob.quality(a) == pytest.approx(unpolished_best)
+
+
+def test_polish_never_breaks_the_budget():
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        L, P = 6, 4
+        lat = rng.uniform(1.0, 3.0, (L, P))
+        keep = rng.uniform(0.0, 1.0, (L, P))
+        budget = float(lat.min(axis=1).sum() + rng.uniform(0.0, 3.0))
+        prob = search.Problem([str(i) for i in range(P)], lat, keep, 10.0, 0.0, budget)
+        a = search.polish(prob, np.argmin(lat, axis=1))
+        assert prob.feasible(a)
+        assert prob.quality(a) >= prob.quality(np.argmin(lat, axis=1)) - 1e-12
