@@ -392,8 +392,7 @@ def run_cosearch(args) -> None:
     ws = lut._Workspace()
     L = lut.profile(shapes, pats_all, [T], reps=10, ws=ws)
     calib = []
-    for i in range(6):
-        asg = lut.random_assignment(len(layers), 400 + i, tuple(pats_all))
+    for asg in lut.stratified_assignments(len(layers), 400) + lut.stratified_assignments(len(layers), 401):
         calib.append((layers, asg, T, lut.measure_sequence(layers, asg, T, reps=3, ws=ws)))
     L.calibrate(calib)
     keep, total = {}, {}

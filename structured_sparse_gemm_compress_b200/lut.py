@@ -73,6 +73,20 @@ def random_assignment(n_layers: int, seed: int, patterns=tuple(PATTERNS)) -> lis
     return [rng.choice(patterns) for _ in range(n_layers)]
 
 
+def stratified_assignments(n_layers: int, seed: int, per_row=tuple(PATTERNS),
+                           tile=tuple(TILE_PATTERNS), fractions=(0.0, 0.25, 0.5, 0.75, 1.0)) -> list[list[str]]:
+    """Calibration assignments whose share of tile-shared layers is set on
+    purpose (one assignment per fraction, layers and patterns drawn at random),
+    so that a per-family term of the calibration is identifiable."""
+    rng = random.Random(seed)
+    out = []
+    for f in fractions:
+        k = round(f * n_layers)
+        tiled = set(rng.sample(range(n_layers), k))
+        out.append([rng.choice(tile) if i in tiled else rng.choice(per_row) for i in range(n_layers)])
+    return out
+
+
 class LatencyLUT:
     """Measured per-launch latency table plus the sequence calibration."""
 

@@ -107,3 +107,11 @@ def test_calibration_recovers_a_per_family_term():
     assert L.predict(layers, asg, 100) == pytest.approx(1.1 * L.raw_sum(layers, asg, 100) + 2.0 + 6.0)
     L2 = lut.LatencyLUT.from_json(L.to_json())
     assert L2.c == pytest.approx(3.0)
+
+
+def test_stratified_assignments_set_the_tile_share():
+    asgs = lut.stratified_assignments(48, 7)
+    assert [lut.n_tile_layers(a) for a in asgs] == [0, 12, 24, 36, 48]
+    for a in asgs:
+        assert len(a) == 48 and set(a) <= set(lut.PATTERNS) | set(lut.TILE_PATTERNS)
+    assert lut.stratified_assignments(48, 7) == asgs                  # seeded
