@@ -282,13 +282,19 @@ def _golden_epilogue():
 
 @pytest.mark.parametrize("case", _golden_epilogue()["cases"], ids=lambda c: c["name"])
 def test_epilogue_hand_cases(case):
-    acc = np.array(case["acc"], dtype=np.int32)
     sc = None if case["scale"] is None else np.array(case["scale"], dtype=np.float32)
     bi = None if case["bias"] is None else np.array(case["bias"], dtype=np.float32)
     exp = np.array(case["expected"])
+    if case.get("path") == "float":  # fp64 accumulator of the FP16/BF16 path, compared in fp64
+        acc = np.array(case["acc"], dtype=np.float64)
+        r = oracle.epilogue(acc, sc, bi, case["act"], case["out"], case["out_scale"])
+        assert np.all(np.abs(r["pre"] - exp) <= case["rel_tol"] * np.abs(exp)), (r["pre"], exp)
+        return
+    acc = np.array(case["acc"], dtype=np.int32)
     if "out_scale_per_case" in case:  # one column at a time, each with its own output scale
         for j, os_ in enumerate(case["out_scale_per_case"]):
-            r = oracle.epilogue(acc[:, j:j + 1], sc, bi, case["act"], case["out"], os_)
+            r = oracle.epilogue(acc[:, j:j + 1], None if sc is None else sc[j:j + 1],
+                                None if bi is None else bi[j:j + 1], case["act"], case["out"], os_)
             assert int(r["q"][0, 0]) == int(exp[0, j])
         return
     r = oracle.epilogue(acc, sc, bi, case["act"], case["out"], case["out_scale"])

@@ -29,7 +29,16 @@ MUTANTS = {
     "bias added before the scale": ("if (scale) v = v * scale[n];\n            if (bias) v = v + bias[n];",
                                     "if (bias) v = v + bias[n];\n            if (scale) v = v * scale[n];"),
     "int8 rounding truncates": ("q[i] = sat_s8((double)rintf(p));", "q[i] = sat_s8((double)truncf(p));"),
-    "GELU drops the 1/2": ("static double gelu_erf(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }",
+    "int8 path: GELU before the bias":
+        ("const double g = gelu_erf((double)v);",
+         "const double g = gelu_erf((double)v - (bias ? bias[n] : 0.0f)) + (bias ? bias[n] : 0.0f);"),
+    "float path: GELU before the bias":
+        ("if (bias) v += (double)bias[n];\n            pre[i] = act == 1 ? gelu_erf(v) : v;",
+         "pre[i] = act == 1 ? gelu_erf(v) : v;\n            if (bias) pre[i] += (double)bias[n];"),
+    "float path: bias before the scale":
+        ("if (scale) v *= (double)scale[n];\n            if (bias) v += (double)bias[n];",
+         "if (bias) v += (double)bias[n];\n            if (scale) v *= (double)scale[n];"),
+    "GELU drops the 1/2":("static double gelu_erf(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }",
                            "static double gelu_erf(double x) { return x * (1.0 + erf(x / sqrt(2.0))); }"),
 }
 
