@@ -156,6 +156,96 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows), "samples_in_timed_region": window}
 
 
+class NvmlSampler:
+    """SM clock, its maximum, power and clock-event reasons of the GPU this
+    process uses (found by PCI bus id), polled by NVML from a thread about
+    every millisecond between ``mark_start`` and ``mark_end``, so even a timed
+    region of a few milliseconds is covered.  Falls back to ``ClockSampler``
+    (nvidia-smi every 50 ms) when NVML is unavailable."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.samples = []
+        self._run = False
+        self._thread = None
+        self._nvml = None
+        self._h = None
+        self._fallback = None
+        self._inside = False
+
+    def __enter__(self):
+        import threading
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(self.dev)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+            self._fallback = ClockSampler(self.dev).__enter__()
+            return self
+        self._run = True
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
+        return self
+
+    def _poll(self):
+        n = self._nvml
+        get_reasons = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            n.nvmlDeviceGetCurrentClocksThrottleReasons
+        while self._run:
+            if self._inside:
+                try:
+                    sm = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+                    rs = get_reasons(self._h)
+                    pw = n.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                    self.samples.append((sm, rs, pw))
+                except Exception:
+                    pass
+                time.sleep(0.0005)
+            else:
+                time.sleep(0.0002)
+
+    def mark_start(self):
+        if self._fallback is not None:
+            return self._fallback.mark_start()
+        self._inside = True
+
+    def mark_end(self):
+        if self._fallback is not None:
+            return self._fallback.mark_end()
+        self._inside = False
+
+    def __exit__(self, *exc):
+        if self._fallback is not None:
+            return self._fallback.__exit__(*exc)
+        self._run = False
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+
+    def summary(self) -> dict:
+        if self._fallback is not None:
+            return self._fallback.summary()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": ["unsampled"],
+                    "samples": 0, "samples_in_timed_region": 0, "source": "nvml"}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({name for _, rs, _ in self.samples for name, bit in self.REASONS if rs & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "power_w_max": round(max(x[2] for x in self.samples), 1),
+                "samples": len(sm), "samples_in_timed_region": len(sm), "source": "nvml, ~1 ms polling"}
+
+
 # --------------------------------------------------------------------------- multi-rank plumbing
 
 
@@ -238,12 +328,17 @@ def roofline_point(l, us: float, pk: dict, out_es: int | None = None, biased: bo
                    gather: bool = False) -> dict:
     """Roofline of one problem: t = max(ops / tensor peak, bytes / HBM peak).
 
-    Tensor peaks derive from the measured bf16 dense peak with NVIDIA's nominal
-    ratios: INT8 dense = 2 x bf16, FP16/BF16 dense = bf16, 2:4-sparse = 2 x dense
-    (1:4, 2:4, 2:8 run on the sparse pipe; 4:8 and N = M on the dense pipe).
+    Tensor peaks: INT8 dense = the INT8 peak measured in the same run
+    (``pk["int8_tops"]``; 2 x the measured bf16 peak, NVIDIA's nominal ratio,
+    when absent), FP16/BF16 dense = the measured bf16 peak, 2:4-sparse = 2 x
+    dense (1:4, 2:4, 2:8 run on the sparse pipe; 4:8 and N = M on the dense
+    pipe).
     gather: tile-shared patterns, whose MMAs run on the dense pipe over the kept
     k only (N/M of the dense-equivalent work)."""
-    dense_peak = pk["bf16_tflops"] * (2.0 if l.dtype == inputs.INT8 else 1.0)
+    if l.dtype == inputs.INT8:
+        dense_peak = pk.get("int8_tops") or pk["bf16_tflops"] * 2.0
+    else:
+        dense_peak = pk["bf16_tflops"]
     sparse = (l.N, l.M) in ((1, 4), (2, 4), (2, 8))
     tc_peak = dense_peak * (2.0 if sparse else 1.0)
     ops = l.dense_ops()
@@ -449,9 +544,12 @@ def run_cosearch(args) -> None:
     print(json.dumps(line), flush=True)
 
 
-def _graph_us(launch, stream, reps: int = 20) -> float:
+def _graph_us(launch, stream, reps: int = 20, replays: int = 5) -> float:
     """Time (us) of one launch: `reps` launches back to back in one CUDA graph,
-    events around the replay, best of three replays."""
+    events around each replay, median over `replays` replays.  Our kernels and
+    cuBLAS's are timed by this same function, so launch overlap (programmatic
+    dependent launch for ours, graph replay for both) and the L2 state (X and
+    W resident across the repeats, Y streaming) are alike."""
     for _ in range(3):
         launch(stream)
     torch.cuda.synchronize()
@@ -463,23 +561,54 @@ def _graph_us(launch, stream, reps: int = 20) -> float:
             launch(cap)
     g.replay()
     torch.cuda.synchronize()
-    best = float("inf")
-    for _ in range(3):
+    ts = []
+    for _ in range(replays):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         g.replay()
         b.record(stream)
         torch.cuda.synchronize()
-        best = min(best, a.elapsed_time(b) * 1e3 / reps)
+        ts.append(a.elapsed_time(b) * 1e3 / reps)
     del g
-    return best
+    return statistics.median(ts)
 
 
-def run_config(name: str, args) -> None:
+def measure_int8_peak(device) -> dict:
+    """Dense INT8 tensor-core peak of this GPU, measured: cuBLAS int8 GEMM
+    (torch._int_mm, int32 out) at 8192^3, CUDA events, best of 20.  The 2:4
+    sparse INT8 peak is taken as twice this (the sparse pipe's nominal ratio)."""
+    n = 8192
+    a = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=device)
+    b = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=device).t()
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(20):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return {"int8_dense_tops": 2.0 * n ** 3 / (best * 1e-3) / 1e12, "how": f"torch._int_mm {n}^3, best of 20"}
+
+
+CONFIG_NAMES = ("single", "vitl", "swin", "mixed1", "mixed256", "int8out", "gather", "gatherl")
+
+
+def measure_config(name: str, args, pk: dict, min_region_ms: float = 200.0, device_index: int = 0) -> dict:
+    """One workload of another configuration, measured on the current device.
+
+    The sequence of its problems runs back to back in one stream, captured as
+    one CUDA graph of `reps` repetitions (no event inside: an event node between
+    kernels serialises them), replayed inside the timed region while the clock
+    sampler runs; reps is raised until the region lasts at least
+    `min_region_ms`.  Per problem, our launch and the same-shape cuBLAS dense
+    GEMM are timed by the same method (``_graph_us``)."""
     import structured_sparse_gemm_compress_b200 as nm
 
-    torch.cuda.set_device(0)
-    pk = peaks()
     if name == "single":
         ls, desc = inputs.single_layer(), "single ViT-B linear, INT8 2:4, T=197, 768->768, int32 out"
     elif name == "vitl":
@@ -533,101 +662,103 @@ def run_config(name: str, args) -> None:
         probs.append((l, W, X, sc, h, Y, call))
     torch.cuda.synchronize()
 
-    def run_all(evs=None):
-        for i, p in enumerate(probs):
-            if evs is not None:
-                evs[i][0].record(stream)
-            p[6](stream)
-            if evs is not None:
-                evs[i][1].record(stream)
+    def run_all(st):
+        for p in probs:
+            p[6](st)
 
-    reps = max(3, args.steps)
     for _ in range(args.warmup):
-        run_all()
+        run_all(stream)
     torch.cuda.synchronize()
-    # The sequence back to back in one stream, captured as one CUDA graph with no
-    # event inside (an event node between kernels serialises them); the
-    # per-problem times come from a second graph with an event pair around
-    # every launch (context: those include the cost of the event nodes).
-    def capture(body):
+
+    def capture(n):
         g = torch.cuda.CUDAGraph()
         cap = torch.cuda.Stream()
         cap.wait_stream(stream)
         with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
-            body(cap)
+            for _ in range(n):
+                run_all(cap)
         g.replay()
         torch.cuda.synchronize()
         return g
 
-    def seq_body(cap):
-        for r in range(reps):
-            for p in probs:
-                p[6](cap)
-
-    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in probs]
-           for _ in range(reps)]
-
-    def per_body(cap):
-        for r in range(reps):
-            for i, p in enumerate(probs):
-                evs[r][i][0].record(cap)
-                p[6](cap)
-                evs[r][i][1].record(cap)
-
-    g = capture(seq_body)
+    # size the timed region: one replay of a single sequence gives the estimate
+    g1 = capture(1)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    g.replay()
+    g1.replay()
     b.record(stream)
     torch.cuda.synchronize()
+    est_ms = max(a.elapsed_time(b), 1e-3)
+    del g1
+    reps = max(3, args.steps, int(min_region_ms / est_ms) + 1)
+    chunk = min(reps, 200)  # graphs of at most 200 sequences, replayed back to back
+    sizes = [chunk] * (reps // chunk) + ([reps % chunk] if reps % chunk else [])
+    built = {n: capture(n) for n in sorted(set(sizes))}
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with NvmlSampler(device_index) as clk:
+        torch.cuda.synchronize()
+        clk.mark_start()
+        a.record(stream)
+        for n in sizes:
+            built[n].replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        clk.mark_end()
     seq_ms = a.elapsed_time(b) / reps
-    del g
-    g = capture(per_body)
-    del g
+    del built
     for h in (p[4] for p in probs):
         if nm.nm_device_status(h) != nm.NM_OK:
             raise RuntimeError(nm.nm_last_error())
     per = []
-    for i, (l, W, X, sc, h, Y, _) in enumerate(probs):
-        us = statistics.median(evs[r][i][0].elapsed_time(evs[r][i][1]) * 1e3 for r in range(reps))
+    for i, (l, W, X, sc, h, Y, call) in enumerate(probs):
+        us = _graph_us(call, stream)
         rp = roofline_point(l, us, pk, 1 if int8out else None, int8out, gather)
+        if not gather:
+            plan = nm.nm_plan_query(h, l.T, scaled=sc is not None)
+            rp["plan"] = {k: plan[k] for k in ("pair", "bn", "splits", "cluster", "grid")}
         if gather:  # the same weight with per-row patterns through nm_spmm (token-major X), same timing
             he = nm.nm_compress(W, l.N, l.M)
             Ye = torch.empty_like(Y)
             rp["per_row_patterns_us"] = round(_graph_us(lambda st: nm.nm_spmm(he, X, Y=Ye, scale=sc, stream=st),
                                                         stream), 2)
-            rp["gather_graph_us"] = round(_graph_us(lambda st: probs[i][6](st), stream), 2)
             he.destroy()
-        # same-shape cuBLAS dense GEMM through torch (context)
+        # same-shape cuBLAS dense GEMM through torch, timed the same way (context)
         if l.dtype == inputs.INT8 and l.T > 16:
-            fn = (lambda X=X, W=W: torch._int_mm(X, W.t()))
+            Wt = W.t()
+            fn = (lambda st, X=X, Wt=Wt: torch._int_mm(X, Wt))
         elif l.dtype != inputs.INT8:
-            fn = (lambda X=X, W=W: torch.matmul(X, W.t()))
+            Wt = W.t()
+            fn = (lambda st, X=X, Wt=Wt: torch.matmul(X, Wt))
         else:
             fn = None
         if fn is not None:
-            for _ in range(3):
-                fn()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(10):
-                fn()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            rp["cublas_dense_us"] = round(e0.elapsed_time(e1) * 100, 2)
+            cb = _graph_us(fn, stream)
+            rp["cublas_dense_us"] = round(cb, 2)
+            rp["vs_cublas"] = round(cb / us, 3)
         rp["problem"] = f"{l.name}/{l.nm}"
         rp["T,K,n_out"] = [l.T, l.K, l.n_out]
         per.append(rp)
     total_ops = sum(l.dense_ops() for l in ls)
     tot_roof = sum(p["roofline_us"] for p in per)
-    sum_us = sum(p["us"] for p in per)
     line = {"config": {"workload": desc}, "metric": "dense-equivalent TOPS over the sequence", "unit": "TOPS",
             "value": total_ops / (seq_ms * 1e-3) / 1e12, "sequence_us": round(seq_ms * 1e3, 2),
-            "sum_of_kernel_us": round(sum_us, 2), "per_problem_note": "an event pair around every launch, separate graph", "roofline_us": round(tot_roof, 2),
-            "roofline_frac": round(tot_roof / (seq_ms * 1e3), 3), "dtype": ls[0].dtype, "data": "synthetic",
-            "launch": "CUDA graph of the sequence", "reps": reps, "per_problem": per}
+            "sum_of_kernel_us": round(sum(p["us"] for p in per), 2),
+            "per_problem_note": ("us: that launch alone, 20 back to back in a CUDA graph (median of 5 replays); "
+                                 "cuBLAS timed the same way"),
+            "roofline_us": round(tot_roof, 2), "roofline_frac": round(tot_roof / (seq_ms * 1e3), 3),
+            "dtype": ls[0].dtype, "data": "synthetic", "launch": "CUDA graph of the sequence", "reps": reps,
+            "clocks": clk.summary(), "per_problem": per}
     if any("cublas_dense_us" in p for p in per):
         line["cublas_dense_sum_us"] = round(sum(p.get("cublas_dense_us", 0.0) for p in per), 2)
+    return line
+
+
+def run_config(name: str, args) -> None:
+    torch.cuda.set_device(0)
+    pk = peaks()
+    pk["int8_tops"] = measure_int8_peak(torch.device("cuda", 0))["int8_dense_tops"]
+    line = measure_config(name, args, pk)
+    line["int8_dense_peak_tops_measured"] = round(pk["int8_tops"], 1)
     print(json.dumps(line), flush=True)
 
 
@@ -644,8 +775,8 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
-    ap.add_argument("--config", default=None, choices=["single", "vitl", "swin", "mixed1", "mixed256", "int8out", "gather",
-                                                       "gatherl", "lut", "search", "cosearch"],
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' blocks in the default line")
+    ap.add_argument("--config", default=None, choices=list(CONFIG_NAMES) + ["lut", "search", "cosearch"],
                     help="measure another workload (one JSON line) instead of the default ViT-B INT8 set")
     ap.add_argument("--only", action="append", default=[],
                     help="restrict to problems like vitb.fc1/2:4 (profiling a single kernel shape)")
@@ -748,7 +879,7 @@ def main() -> None:
         torch.cuda.synchronize()
 
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with NvmlSampler(local_rank) as clk:
         barrier()
         torch.cuda.synchronize()
         clk.mark_start()
@@ -781,43 +912,6 @@ def main() -> None:
     pk = peaks()
     achieved = spmm_bytes / (ms_local * 1e-3) / 1e9
 
-    # Per-launch breakdown (context, not the timed region): one more pass of the
-    # step in its own graph with an event pair around every SpMM and re-pack.
-    pl = [[torch.cuda.Event(enable_timing=True, external=not args.no_graph) for _ in range(2)] for _ in ls]
-    pk_ev = [torch.cuda.Event(enable_timing=True, external=not args.no_graph) for _ in range(2)]
-
-    def breakdown_pass(st, ps):
-        ps.wait_stream(st)
-        pk_ev[0].record(ps)
-        for i, l in enumerate(ls):
-            nm.nm_recompress(handles[i], devb[l.name]["W"], stream=ps)
-        pk_ev[1].record(ps)
-        st.wait_stream(ps)
-        for i, l in enumerate(ls):
-            d = devb[l.name]
-            pl[i][0].record(st)
-            nm.nm_spmm(handles[i], d["X"], Y=Ys[i], scale=d["s"], stream=st)
-            pl[i][1].record(st)
-
-    if args.no_graph:
-        breakdown_pass(stream, pack_stream)
-    else:
-        g2 = torch.cuda.CUDAGraph()
-        cap, cap_pack = torch.cuda.Stream(), torch.cuda.Stream()
-        cap.wait_stream(stream)
-        with torch.cuda.graph(g2, stream=cap, capture_error_mode="thread_local"):
-            breakdown_pass(cap, cap_pack)
-        g2.replay()
-        torch.cuda.synchronize()
-        g2.replay()
-        del g2
-    torch.cuda.synchronize()
-    per_layer = {}
-    for i, l in enumerate(ls):
-        t = pl[i][0].elapsed_time(pl[i][1])
-        per_layer[f"{l.name}/{l.nm}"] = {"us": round(t * 1e3, 2), "dense_eq_tops": round(l.dense_ops() / t / 1e9, 1),
-                                        "gbs": round(alg_bytes(l) / t / 1e6, 1)}
-    pack_us = 1e3 * pk_ev[0].elapsed_time(pk_ev[1])
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "spmm_vitb_int8_traffic.json")
     if os.path.exists(tfile):
@@ -825,23 +919,36 @@ def main() -> None:
         if tj.get("kernel_source_sha") == _kernel_sha():
             traffic = tj.get("bytes_per_launch")
 
-    # cuBLAS dense INT8 GEMM of the same shapes (context: torch._int_mm -> int32).
-    cublas = {}
+    # Per-layer context (not the timed region), rank 0: every problem alone and
+    # cuBLAS's dense int8 GEMM of the same shape (torch._int_mm, int32 out),
+    # both timed by _graph_us (20 back-to-back launches in a CUDA graph, median
+    # of 5 replays), plus the measured INT8 tensor peak.
+    per_layer, cublas, pack_us, int8_peak = {}, {}, None, None
     if rank == 0:
+        int8_peak = measure_int8_peak(dev)
+        pk["int8_tops"] = int8_peak["int8_dense_tops"]
         for name in sorted({x.name for x in ls}):
-            l = next(x for x in ls if x.name == name)
-            Xd, Wd = devb[name]["X"], devb[name]["W"]
-            Wt = Wd.t()
-            for _ in range(3):
-                torch._int_mm(Xd, Wt)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(10):
-                torch._int_mm(Xd, Wt)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            t = e0.elapsed_time(e1) / 10
-            cublas[name] = {"us": round(t * 1e3, 2), "dense_tops": round(l.dense_ops() / t / 1e9, 1)}
+            Xd, Wt = devb[name]["X"], devb[name]["W"].t()
+            cublas[name] = _graph_us(lambda st, Xd=Xd, Wt=Wt: torch._int_mm(Xd, Wt), stream)
+        for i, l in enumerate(ls):
+            d = devb[l.name]
+            us = _graph_us(lambda st, i=i, d=d: nm.nm_spmm(handles[i], d["X"], Y=Ys[i], scale=d["s"], stream=st),
+                           stream)
+            rp = roofline_point(l, us, pk)
+            rp["hbm_frac"] = round(alg_bytes(l) / (us * 1e-6) / 1e9 / pk["hbm_gbs"], 3)
+            rp["cublas_int8_dense_us"] = round(cublas[l.name], 2)
+            rp["vs_cublas"] = round(cublas[l.name] / us, 3)
+            plan = nm.nm_plan_query(handles[i], l.T, scaled=True)
+            rp["plan"] = {k: plan[k] for k in ("pair", "bn", "splits", "cluster", "grid")}
+            per_layer[f"{l.name}/{l.nm}"] = rp
+
+        def all_packs(st):
+            for i, l in enumerate(ls):
+                nm.nm_recompress(handles[i], devb[l.name]["W"], stream=st)
+
+        pack_us = _graph_us(all_packs, stream, reps=5)
+        cublas = {k: {"us": round(v, 2), "dense_tops": round(
+            next(x for x in ls if x.name == k).dense_ops() / v / 1e6, 1)} for k, v in cublas.items()}
 
     # End to end through the public API with host buffers: every step copies its
     # inputs (weights, activations, scales) from pinned host memory and reads
@@ -911,10 +1018,27 @@ def main() -> None:
         "spmm_launch_us_avg": 1e3 * ms_local / (args.steps * len(ls)),
         "pack_us_per_step": pack_us,
         "pack_overlapped": True,
-        "per_layer_note": "one untimed extra pass, an event pair around every launch",
+        "int8_dense_peak_tops_measured": None if int8_peak is None else round(int8_peak["int8_dense_tops"], 1),
+        "per_layer_note": ("each problem alone and cuBLAS's int8 GEMM of the same shape, both as 20 back-to-back "
+                           "launches in a CUDA graph (median of 5 replays); hbm_frac = algorithmic bytes / time / "
+                           "measured HBM; frac = roofline (max of HBM and tensor time, INT8 peak measured) / time"),
         "per_layer": per_layer,
         "cublas_int8_dense": cublas,
     }
+    if not args.no_extras:
+        # The other workloads, each with its own clock record (context for the
+        # tensor-bound FP16 set, the small-token adaptive split-K and the
+        # Swin stages): the sequence timed as one graph, per problem ours and
+        # cuBLAS's timed the same way.
+        import types
+        eargs = types.SimpleNamespace(steps=3, warmup=3)
+        extras = {}
+        for cname in ("vitl", "mixed1", "single", "swin", "mixed256"):
+            r = measure_config(cname, eargs, pk, min_region_ms=200.0, device_index=local_rank)
+            for p in r["per_problem"]:
+                p.pop("T,K,n_out", None)
+            extras[cname] = r
+        line["configs"] = extras
     print(json.dumps(line), flush=True)
 
 

@@ -83,11 +83,16 @@ nm_status nm_compress(const void* W_dev, int64_t n_out, int64_t k, nm_dtype dt, 
  * which can synchronise the device and take a process-wide lock.
  *
  * Arguments, layouts, rounding and results are those of nm_spmm.  The
- * difference is where the split-K scratch (partial tiles and per-tile arrival
- * counters) lives: in one fixed array inside the library, 4 MiB of partials
- * plus 1024 counters.  Every GPU that loads the library holds that array until
- * the process exits.  This call never calls cudaMalloc, cudaFree or any
- * allocating routine.
+ * difference is where the scratch of a global-memory split-K (partial tiles
+ * and per-tile arrival counters) lives: in one fixed array inside the
+ * library, 4 MiB of partials plus 1024 counters.  Every GPU that loads the
+ * library holds that array until the process exits.  This call never calls
+ * cudaMalloc, cudaFree or any allocating routine.
+ *   - The planner's own plans never use the array: they either do not split
+ *     k or reduce the splits on chip (see nm_spmm).  Only a global-memory
+ *     split forced through the environment (NMSPMM_FORCE_SPLITK with
+ *     NMSPMM_SPLIT_GLOBAL=1, or more than 8 splits) uses it, and only then do
+ *     the size limit and the race below apply.
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (set-up, once per device, with that device
  *     current); make that first call before any stream capture.
@@ -127,12 +132,17 @@ nm_status nm_recompress(nm_handle* h, const void* W_dev, void* stream);
  *           Must be 16-byte aligned and must not overlap X.
  * scale_dev float32 [n_out] or NULL.
  * T         >= 0; T == 0 is a no-op returning NM_OK.
- * The tile shape and split-K factor are chosen per (T, k, n_out, N:M, dtype)
- * so that small token counts still occupy every SM.  When split-K is used the
- * handle's workspace is used: calls on one handle must not overlap on the GPU
- * (the same rule as a library handle with a workspace).  The first call that
- * needs split-K allocates that workspace (make it before any stream capture).
- * Never synchronises.
+ * The kernel, token tile and split-K factor are chosen per (T, k, n_out,
+ * N:M, dtype) so that small token counts still occupy the SMs (section 4.1,
+ * mechanism 3; nm_plan_query reports the choice).  A split chosen by the
+ * planner puts the k-splits of one output tile on the CTAs of one
+ * thread-block cluster, which sum their partial tiles through distributed
+ * shared memory: no workspace, no allocation.  A global-memory split-K
+ * (forced through the environment: NMSPMM_FORCE_SPLITK with
+ * NMSPMM_SPLIT_GLOBAL=1, or more than 8 splits) uses the handle's workspace:
+ * calls on one handle must then not overlap on the GPU, and the first such
+ * call allocates the workspace (after a device synchronisation; make it
+ * before any stream capture).  Otherwise never synchronises.
  */
 nm_status nm_spmm(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
                   const float* scale_dev, void* stream);
@@ -235,9 +245,9 @@ nm_status nm_compress_tile(const void* W_dev, int64_t n_out, int64_t k, nm_dtype
  * scale_dev float32 [n_out] or NULL.
  * T         >= 0; T == 0 is a no-op.
  * The default plan never splits k, so the call allocates nothing and never
- * synchronises; a split-K plan forced through NMSPMM_FORCE_SPLITK uses the
- * handle's workspace under the rules of nm_spmm (the first such call
- * allocates it, after a device synchronisation).
+ * synchronises; a split-K plan forced through NMSPMM_FORCE_SPLITK reduces in
+ * global memory and uses the handle's workspace under the rules of nm_spmm
+ * (the first such call allocates it, after a device synchronisation).
  */
 nm_status nm_spmm_gather(const nm_handle* h, const void* Xt_dev, int64_t ldx, int64_t T, void* Y_dev,
                          const float* scale_dev, void* stream);
@@ -271,6 +281,24 @@ nm_status nm_decompress(const nm_handle* h, void* W_dev_out, void* stream);
  */
 nm_status nm_export(const nm_handle* h, void* values_host, uint8_t* idx_host);
 nm_status nm_export_sizes(const nm_handle* h, size_t* values_bytes, size_t* idx_bytes);
+
+/*
+ * nm_plan_query -- the launch plan nm_spmm (scaled != 0: with a scale; the
+ * INT8 fp32-output kernels) would use for T tokens on the current device,
+ * without launching anything (section 4.1, mechanism 3, adaptive
+ * parallelism).  For a handle from nm_compress_tile it is nm_spmm_gather's
+ * plan.  Environment overrides (NMSPMM_FORCE_*) apply as they would to the
+ * call.  T > 0, else NM_ERR_INVALID.
+ */
+typedef struct nm_plan_info {
+  int pair;     /* 1: two-SM kernel (M = 256 per MMA, grid counts CTA pairs) */
+  int bn;       /* token tile (MMA N) */
+  int splits;   /* k-splits per output tile (1: none) */
+  int cluster;  /* 1: the splits of a tile are one cluster, reduced on chip */
+  int grid;     /* CTAs launched (CTA pairs for the two-SM kernel) */
+  int units;    /* (tile, split) work units */
+} nm_plan_info;
+nm_status nm_plan_query(const nm_handle* h, int64_t T, int scaled, nm_plan_info* out);
 
 /* nm_query -- shape and format of a handle; any output pointer may be NULL. */
 nm_status nm_query(const nm_handle* h, int64_t* n_out, int64_t* k, int* N, int* M, nm_dtype* dt);

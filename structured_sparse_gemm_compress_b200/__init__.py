@@ -26,7 +26,13 @@ _ELEM = {NM_INT8: torch.int8, NM_FP16: torch.float16, NM_BF16: torch.bfloat16}
 # Every symbol include/nmspmm.h declares.
 EXPORTS = ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_ex", "nm_spmm_gather",
            "nm_spmm_gather_ex", "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
-           "nm_device_status", "nm_destroy", "nm_last_error", "nm_version", "nm_test_spmm_skip_stage")
+           "nm_plan_query", "nm_device_status", "nm_destroy", "nm_last_error", "nm_version", "nm_test_spmm_skip_stage")
+
+
+class NMPlanInfo(ctypes.Structure):
+    """nm_plan_info of include/nmspmm.h."""
+    _fields_ = [("pair", ctypes.c_int), ("bn", ctypes.c_int), ("splits", ctypes.c_int),
+                ("cluster", ctypes.c_int), ("grid", ctypes.c_int), ("units", ctypes.c_int)]
 
 
 class NMError(RuntimeError):
@@ -61,6 +67,7 @@ def lib() -> ctypes.CDLL:
         L.nm_export_sizes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
         L.nm_query.argtypes = [vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i32),
                                ctypes.POINTER(i32), ctypes.POINTER(i32)]
+        L.nm_plan_query.argtypes = [vp, i64, i32, ctypes.POINTER(NMPlanInfo)]
         L.nm_device_status.argtypes = [vp]
         L.nm_destroy.argtypes = [vp]
         L.nm_destroy.restype = None
@@ -69,7 +76,7 @@ def lib() -> ctypes.CDLL:
         for name in ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_gather",
                      "nm_spmm_gather_ex", "nm_spmm_noalloc",
                      "nm_test_spmm_skip_stage", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
-                     "nm_device_status"):
+                     "nm_plan_query", "nm_device_status"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -313,6 +320,13 @@ def nm_query(h: NMHandle) -> dict:
     _check(lib().nm_query(h.raw, ctypes.byref(n), ctypes.byref(k), ctypes.byref(N), ctypes.byref(M),
                           ctypes.byref(dt)))
     return {"n_out": n.value, "k": k.value, "N": N.value, "M": M.value, "dtype": dt.value}
+
+
+def nm_plan_query(h: NMHandle, T: int, scaled: bool = False) -> dict:
+    """The launch plan the SpMM call would use for T tokens (kernel, token tile, splits, cluster, grid)."""
+    info = NMPlanInfo()
+    _check(lib().nm_plan_query(h.raw, int(T), int(bool(scaled)), ctypes.byref(info)))
+    return {f: getattr(info, f) for f, _ in NMPlanInfo._fields_}
 
 
 def nm_device_status(h: NMHandle) -> int:

@@ -201,6 +201,65 @@ int out_code(const nm_handle* h, bool scaled) {
   return h->dt == nm::DT_F16 ? nm::OUT_F16 : nm::OUT_BF16;
 }
 
+// Small-token model of one streaming launch (us), fitted on B200 to a sweep of
+// forced (token tile, split) plans over the ViT-B INT8 shapes at T = 16 .. 788
+// (CUDA graphs of back-to-back launches; within ~5 % of every point):
+//   waves x (start + epilogue + reduction + load), where
+//   load = max(k-blocks per CTA x per-k-block time at one SM's L2 rate,
+//              operand bytes of the resident tiles / aggregate L2 rate),
+// the reduction (cluster launch, two cluster barriers, parked partials read
+// through distributed shared memory) paid only when k is split.
+struct SmallTModel {
+  double start = 2.7;          // launch, first operand latency, completion
+  double per_kb = 0.24;        // one k-block at one SM's L2 rate, plus per token column:
+  double per_kb_tok = 0.0006;
+  double epi_tok = 0.004;      // epilogue per token column
+  double red = 1.2;            // on-chip reduction, plus per token column:
+  double red_tok = 0.012;
+  double l2_bytes_per_us = 10.0e6;  // aggregate L2 -> SM operand rate (~10 TB/s)
+};
+
+double small_t_cost(const nm_handle* h, int64_t T, int sms, int bn, int S) {
+  const SmallTModel m;
+  const int64_t tiles = (int64_t)h->n_ct * ((T + bn - 1) / bn);
+  const int kbs = (h->n_kb + S - 1) / S;
+  int64_t cap = sms;  // tiles resident at once: one per SM, or one per resident cluster
+  if (S > 1) {
+    const int c = nm::stream_max_clusters(S);
+    if (c <= 0) return 1e300;
+    cap = c;
+  }
+  const int64_t waves = (tiles + cap - 1) / cap;
+  const double stage = (double)nm::chunk_bytes(h->dt, h->img) + 256.0 * bn;  // packed chunk + X rows
+  const double load = std::max(kbs * (m.per_kb + m.per_kb_tok * bn),
+                               (double)std::min(tiles, cap) * h->n_kb * stage / m.l2_bytes_per_us);
+  double t = m.start + m.epi_tok * bn + load;
+  if (S > 1) t += m.red + m.red_tok * bn;
+  return (double)waves * t;
+}
+
+// For a shape whose unsplit tiles leave SMs idle: keeps the streaming rule's
+// token tile unsplit unless, by the model above, some (token tile, split > 1)
+// is clearly faster; then sets both.  (Measured: at T <= 64 the K = 3072 ViT-B
+// layer drops from 5.8 to 4.8 us with 6 splits of 32-token tiles; K = 768
+// layers, whose 3 k-blocks leave nothing to split, stay unsplit.)
+void choose_cluster_split(const nm_handle* h, int64_t T, int sms, int forced_bn, nm::Plan* p, int* splits) {
+  double best = small_t_cost(h, T, sms, p->bn, 1);
+  for (int bn : {32, 64, 128}) {
+    if (forced_bn && bn != forced_bn) continue;
+    for (int S = 2; S <= std::min(nm::kMaxClusterSplit, h->n_kb); ++S) {
+      const int kps = (h->n_kb + S - 1) / S;
+      if ((h->n_kb + kps - 1) / kps != S) continue;  // every split owns >= 1 k-block
+      const double c = small_t_cost(h, T, sms, bn, S);
+      if (c < best * 0.95) {  // a clear win only
+        best = c;
+        p->bn = bn;
+        *splits = S;
+      }
+    }
+  }
+}
+
 // Adaptive parallelism: pick the kernel (CTA pair or single SM), the token tile
 // and the split-K factor for this shape (rules and their measurements below).
 nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
@@ -298,22 +357,32 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
       p.bn = bn;
     }
   }
-  p.n_tt = (int)((T + p.bn - 1) / p.bn);
-  const int64_t tiles = (int64_t)h->n_ct * p.n_tt;
   int splits = 1;
   if (forced_split > 0) {
     splits = forced_split;
+  } else if (env_int("NMSPMM_CSPLIT", 1) != 0) {
+    // Small token counts: too few tiles to occupy the SMs.  Split k over the
+    // CTAs of a cluster, which sum their partials on chip (no workspace), when
+    // the model below says that beats the unsplit tile.
+    const int64_t tiles0 = (int64_t)h->n_ct * ((T + p.bn - 1) / p.bn);
+    if (tiles0 < sms) choose_cluster_split(h, T, sms, forced_bn, &p, &splits);
   }
-  // No split-K by default: measured on B200, the partial round trip (write,
-  // arrival counter, last-arriver reduction) costs more than the idle SMs it
-  // fills, down to 6 tiles on 148 SMs (ViT-B qkv/proj/fc1 at T = 16, 64, 197:
-  // 3.7-3.8 us unsplit against 5.8-13 us split; fc2 at T = 64: 6.9 vs 8.3 us).
-  // The split-K path stays available (NMSPMM_FORCE_SPLITK) and tested.
+  p.n_tt = (int)((T + p.bn - 1) / p.bn);
+  const int64_t tiles = (int64_t)h->n_ct * p.n_tt;
   splits = std::max(1, std::min(splits, h->n_kb));
   p.kb_per_split = (h->n_kb + splits - 1) / splits;
   p.splits = (h->n_kb + p.kb_per_split - 1) / p.kb_per_split;  // every split owns >= 1 k-block
   p.units = (int)(tiles * p.splits);
   p.grid = std::min(p.units, sms);
+  // Splits of one tile form a cluster and reduce through distributed shared
+  // memory (one unit per CTA: the grid is every unit), unless the global
+  // workspace reduction is asked for (NMSPMM_SPLIT_GLOBAL=1) or the split is
+  // wider than a portable cluster.
+  if (p.splits > 1 && p.splits <= nm::kMaxClusterSplit && env_int("NMSPMM_SPLIT_GLOBAL", 0) == 0 &&
+      nm::stream_max_clusters(p.splits) > 0) {
+    p.cluster = 1;
+    p.grid = p.units;
+  }
   return p;
 }
 
@@ -400,8 +469,44 @@ nm_status reject_tile(const nm_handle* h) {
   return NM_OK;
 }
 
+// Split-K scratch supplied by the caller instead of the handle's workspace
+// (nm_spmm_noalloc): partial tiles and arrival counters with their capacities.
+struct SplitScratch {
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int* cnt = nullptr;
+  int cnt_len = 0;
+};
+
+// Workspace of a global-memory split-K launch of plan `p`: the handle's (grown
+// on demand) or the caller's `ext` (never grown: too small is an error).  The
+// tiles' arrival counters are cleared on the stream before the launch: a
+// launch that gave up a bounded wait can leave them part-counted.
+nm_status split_workspace(nm_handle* h, const nm::Plan& p, const SplitScratch* ext, cudaStream_t s,
+                          nm::SpmmArgs* a) {
+  const int tiles = h->n_ct * p.n_tt;
+  if (ext) {
+    const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
+    if (need > ext->ws_bytes || tiles > ext->cnt_len)
+      return fail(NM_ERR_UNSUPPORTED,
+                  "this shape needs %zu bytes of split-K scratch for %d tiles; the allocation-free entry point "
+                  "holds at most %zu bytes and %d tiles (use nm_spmm)",
+                  need, tiles, ext->ws_bytes, ext->cnt_len);
+    a->ws = ext->ws;
+    a->cnt = ext->cnt;
+  } else {
+    nm_status st = ensure_split_workspace(h, p);
+    if (st != NM_OK) return st;
+    a->ws = h->d_ws;
+    a->cnt = h->d_cnt;
+  }
+  cudaError_t e = cudaMemsetAsync(a->cnt, 0, (size_t)tiles * sizeof(int), s);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "clear the split-K counters");
+}
+
 nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, const float* scale, void* stream,
-                    int inject_skip, unsigned long long timeout_ns, const EpiReq* ep = nullptr) {
+                    int inject_skip, unsigned long long timeout_ns, const EpiReq* ep = nullptr,
+                    const SplitScratch* ext = nullptr) {
   g_err.clear();
   nm_status st = check_handle(hc);
   if (st != NM_OK) return st;
@@ -450,10 +555,11 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   // timeline builds only: device buffer of grid * kTraceStride int64 given as an integer address
   if (const char* tp = getenv("NMSPMM_TRACE_PTR")) a.trace = reinterpret_cast<long long*>(strtoull(tp, nullptr, 0));
 #endif
-  if (p.splits > 1) {
-    if ((st = ensure_split_workspace(h, p)) != NM_OK) return st;
-    a.ws = h->d_ws;
-    a.cnt = h->d_cnt;
+  a.prefetch = std::max(0, std::min(2, env_int("NMSPMM_PREFETCH", 1)));
+  if (p.cluster) {
+    a.csplit = 1;  // partials summed on chip: no workspace
+  } else if (p.splits > 1) {
+    if ((st = split_workspace(h, p, ext, (cudaStream_t)stream, &a)) != NM_OK) return st;
   }
   int oes, oty;
   out_type(h, scale != nullptr, &oes, &oty);
@@ -463,7 +569,8 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   // Direct stores measured faster than staged TMA stores (they keep the TMA unit
   // for operand loads); the TMA-store epilogue remains selectable.
   a.tma_store = 0;
-  if (env_int("NMSPMM_TMA_STORE", 0) && a.out_ty < 0) a.tma_store = make_y_map(h, Y, T, oes, oty, ych, &st) ? 1 : 0;
+  if (env_int("NMSPMM_TMA_STORE", 0) && a.out_ty < 0 && !p.cluster)
+    a.tma_store = make_y_map(h, Y, T, oes, oty, ych, &st) ? 1 : 0;
   if (st != NM_OK) return st;
   cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "launch SpMM kernel");
@@ -746,11 +853,7 @@ nm_status gather_impl(const nm_handle* hc, const void* Xt, int64_t ldx, int64_t 
   a.bias = ep ? ep->bias : nullptr;
   a.act = ep ? ep->act : nm::ACT_NONE;
   a.out_scale = ep ? ep->out_scale : 1.0f;
-  if (p.splits > 1) {
-    if ((st = ensure_split_workspace(h, p)) != NM_OK) return st;
-    a.ws = h->d_ws;
-    a.cnt = h->d_cnt;
-  }
+  if (p.splits > 1 && (st = split_workspace(h, p, nullptr, (cudaStream_t)stream, &a)) != NM_OK) return st;
   cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch SpMM kernel");
 }
@@ -791,6 +894,22 @@ nm_status nm_export(const nm_handle* h, void* values_host, uint8_t* idx_host) {
   return NM_OK;
 }
 
+nm_status nm_plan_query(const nm_handle* h, int64_t T, int scaled, nm_plan_info* out) {
+  g_err.clear();
+  nm_status st = check_handle(h);
+  if (st != NM_OK) return st;
+  if (!out) return fail(NM_ERR_INVALID, "null output");
+  if (T <= 0 || T > INT32_MAX) return fail(NM_ERR_INVALID, "T must be in [1, 2^31-1] (got %lld)", (long long)T);
+  const nm::Plan p = make_plan(h, T, num_sms(h->device), scaled != 0);
+  out->pair = p.pair;
+  out->bn = p.bn;
+  out->splits = p.splits;
+  out->cluster = p.cluster;
+  out->grid = p.grid;
+  out->units = p.units;
+  return NM_OK;
+}
+
 nm_status nm_query(const nm_handle* h, int64_t* n_out, int64_t* k, int* N, int* M, nm_dtype* dt) {
   g_err.clear();
   if (!h) return fail(NM_ERR_INVALID, "null handle");
@@ -818,75 +937,20 @@ nm_status nm_device_status(const nm_handle* h) {
   return fail(NM_ERR_TIMEOUT, "a kernel gave up a bounded wait (%s)", (word >= 1 && word <= 4) ? where[word] : "?");
 }
 
-nm_status nm_spmm_noalloc(const nm_handle* hc, const void* X, int64_t T, void* Y, const float* scale,
+nm_status nm_spmm_noalloc(const nm_handle* h, const void* X, int64_t T, void* Y, const float* scale,
                           void* stream) {
   g_err.clear();
-  nm_status st = check_handle(hc);
+  nm_status st = check_handle(h);
   if (st != NM_OK) return st;
-  if ((st = reject_tile(hc)) != NM_OK) return st;
-  nm_handle* h = const_cast<nm_handle*>(hc);  // only the tensor-map cache (host memory) changes
   void* scratch = nullptr;
   st = noalloc_scratch(h->device, &scratch);  // first call on this device: address lookup
   if (st != NM_OK) return st;
-  if (T < 0) return fail(NM_ERR_INVALID, "T must be >= 0 (got %lld)", (long long)T);
-  if (T == 0) return NM_OK;
-  if (!X || !Y) return fail(NM_ERR_INVALID, "null X or Y");
-  if (T > INT32_MAX) return fail(NM_ERR_UNSUPPORTED, "T above 2^31-1");
-  const int es = nm::elem_bytes(h->dt);
-  if (!aligned(X, 16) || !aligned(Y, 16)) return fail(NM_ERR_INVALID, "X and Y must be 16-byte aligned");
-  if ((h->k * es) % 16 != 0)
-    return fail(NM_ERR_UNSUPPORTED, "k * sizeof(dtype) must be a multiple of 16 bytes (k=%lld)", (long long)h->k);
-  if (scale && !aligned(scale, 4)) return fail(NM_ERR_INVALID, "scale must be 4-byte aligned");
-  const size_t ybytes = (size_t)T * h->n_out * ((h->dt == nm::DT_I8) ? 4 : 2);
-  const size_t xbytes = (size_t)T * h->k * es;
-  const uintptr_t xs = (uintptr_t)X, ys = (uintptr_t)Y;
-  if (xs < ys + ybytes && ys < xs + xbytes) return fail(NM_ERR_INVALID, "Y overlaps X");
-
-  const nm::Plan p = make_plan(h, T, num_sms(h->device), scale != nullptr);
-  st = make_x_map(h, X, T, p.pair ? p.bn / 2 : p.bn);
-  if (st != NM_OK) return st;
-  nm::SpmmArgs a{};
-  a.bpack = h->d_bpack;
-  a.Y = Y;
-  a.scale = scale;
-  a.err = h->d_err;
-  a.T = (int)T;
-  a.n_out = (int)h->n_out;
-  a.n_kb = h->n_kb;
-  a.n_ct = h->n_ct;
-  a.n_tt = p.n_tt;
-  a.splits = p.splits;
-  a.kb_per_split = p.kb_per_split;
-  a.units = p.units;
-  a.timeout_ns = 1000000000ull;
-  a.inject_skip = -1;
-  a.w_tma = h->has_tmw;
-  if (p.splits > 1) {
-    const int tiles = h->n_ct * p.n_tt;
-    const size_t need = (size_t)tiles * p.splits * p.bn * nm::kRows * 4;
-    if (need > kNoAllocPartialBytes || tiles > kNoAllocCounters)
-      return fail(NM_ERR_UNSUPPORTED,
-                  "this shape needs %zu bytes of split-K scratch for %d tiles; the allocation-free entry point "
-                  "holds at most %zu bytes and %d tiles (use nm_spmm)",
-                  need, tiles, kNoAllocPartialBytes, kNoAllocCounters);
-    a.ws = scratch;
-    a.cnt = reinterpret_cast<int*>(static_cast<unsigned char*>(scratch) + kNoAllocPartialBytes);
-    // The array keeps the previous call's contents: the counters must start at zero.
-    cudaError_t e = cudaMemsetAsync(a.cnt, 0, (size_t)tiles * sizeof(int), (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "clear the split-K counters");
-  }
-  int oes, oty;
-  out_type(h, scale != nullptr, &oes, &oty);
-  const int wcols = p.bn / nm::epw_for(false);  // token columns per epilogue warp; the TMA-store box
-  const int ych = p.pair ? (wcols % 32 == 0 ? 32 : wcols % 16 == 0 ? 16 : 8)
-                         : (wcols % 32 == 0 ? 32 : (wcols % 8 == 0 && wcols <= 96) ? wcols : 8);
-  // Direct stores measured faster than staged TMA stores (they keep the TMA unit
-  // for operand loads); the TMA-store epilogue remains selectable.
-  a.tma_store = 0;
-  if (env_int("NMSPMM_TMA_STORE", 0)) a.tma_store = make_y_map(h, Y, T, oes, oty, ych, &st) ? 1 : 0;
-  if (st != NM_OK) return st;
-  cudaError_t e = nm::launch_spmm(h, &h->tm, &h->tmy, p, a, (cudaStream_t)stream);
-  return e == cudaSuccess ? NM_OK : cuda_fail(e, "launch SpMM kernel");
+  SplitScratch ext;
+  ext.ws = scratch;
+  ext.ws_bytes = kNoAllocPartialBytes;
+  ext.cnt = reinterpret_cast<int*>(static_cast<unsigned char*>(scratch) + kNoAllocPartialBytes);
+  ext.cnt_len = kNoAllocCounters;
+  return spmm_impl(h, X, T, Y, scale, stream, -1, 1000000000ull, nullptr, &ext);
 }
 
 void nm_destroy(nm_handle* h) {

@@ -66,6 +66,8 @@ struct Plan {
   int grid = 1;       // persistent CTAs
   int xkb = 0;        // > 0: X-stationary mode holding this many k-blocks of X resident
   int pair = 0;       // 1: CTA-pair kernel (M = 256 per MMA); grid counts pairs
+  int cluster = 0;    // 1: the splits of a tile are the CTAs of one cluster (grid = units, one unit
+                      //    per CTA) and their partials are summed through distributed shared memory
 };
 
 // Epilogue warps per TMEM lane quarter (each owns BN / epw token columns of a
@@ -107,6 +109,12 @@ struct SpmmArgs {
   long long ldx = 0;
   int gather_tma = 0;
   long long* trace;   // timeline buffer, only written by builds compiled with NM_TRACE
+  // Split-K reduced on chip (streaming kernel, splits > 1): the `splits` CTAs of
+  // a cluster are the splits of one tile, one unit per CTA; ws and cnt unused.
+  int csplit = 0;
+  // Before waiting for the previous kernel of the stream, hint into L2 the
+  // first unit's weight chunks (1) and also its activation boxes (2); 0: none.
+  int prefetch = 0;
 };
 
 // Timeline trace layout (builds with NM_TRACE): per CTA kTraceStride int64
@@ -121,6 +129,10 @@ cudaError_t launch_decompress(const nm_handle* h, void* Wout, cudaStream_t s);
 cudaError_t launch_compress_tile(const nm_handle* h, const void* W, cudaStream_t s);
 // Resident CTA pairs for the pair kernel of this (dtype, image, token tile, output) or <= 0.
 int pair_max_clusters(int dt, int img, int bn, int out);
+// Clusters of `size` one-SM streaming CTAs that can be resident at once (<= 0: none).
+int stream_max_clusters(int size);
+// Largest cluster the on-chip split-K uses (portable cluster size).
+constexpr int kMaxClusterSplit = 8;
 cudaError_t launch_spmm(const nm_handle* h, const CUtensorMap* tmX, const CUtensorMap* tmY, const Plan& p,
                         const SpmmArgs& a, cudaStream_t s);
 

@@ -365,6 +365,84 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]) {
   tmem_ld_run<N>(taddr, r);
 }
 
+__device__ __forceinline__ uint32_t out_bits(int32_t v) { return (uint32_t)v; }
+__device__ __forceinline__ uint32_t out_bits(float v) { return __float_as_uint(v); }
+__device__ __forceinline__ uint32_t out_bits(__half v) { return (uint32_t)__half_as_ushort(v); }
+__device__ __forceinline__ uint32_t out_bits(__nv_bfloat16 v) { return (uint32_t)__bfloat16_as_ushort(v); }
+
+// On-chip split-K reduction.  The S = a.splits CTAs of a cluster computed the
+// S k-ranges of one tile and parked their partial tiles in their own shared
+// memory at `xb_local` ([BN token columns][128 channels], 32-bit).  This CTA
+// (cluster rank w.z) finishes the token columns j with j % S == w.z: it reads
+// the S partials of a column through distributed shared memory, sums them in
+// split order (so fp32 sums do not depend on timing), applies the output stage
+// and stores.  Each thread owns four consecutive channels, so a warp covers the
+// tile's 128 channels of one token with 16-byte reads and stores.
+template <int DT, int BN, int OUT, int EPI_WARPS>
+__device__ __forceinline__ void csplit_reduce(const SpmmArgs& a, const Unit& w, uint32_t xb_local, int ew,
+                                              int lane) {
+  constexpr bool EPI = (OUT & kOutEpi) != 0;
+  const int S = a.splits;
+  uint32_t src[kMaxClusterSplit];
+#pragma unroll
+  for (int z = 0; z < kMaxClusterSplit; ++z) src[z] = z < S ? mapa_shared(xb_local, (uint32_t)z) : 0u;
+  const int chl = 4 * lane;
+  const int ch = w.ct * kRows + chl;
+  const bool vec = (a.n_out & 3) == 0;  // whole, aligned 4-channel groups
+  const bool has_scale = a.scale != nullptr;
+  float sc[4], bi[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool ok = ch + i < a.n_out;
+    sc[i] = (has_scale && ok) ? __ldg(a.scale + ch + i) : 1.0f;
+    bi[i] = (EPI && a.bias && ok) ? __ldg(a.bias + ch + i) : 0.0f;
+  }
+  if (ch >= a.n_out) return;
+#pragma unroll 1
+  for (int j = w.z + S * ew; j < BN; j += S * EPI_WARPS) {
+    const int t = w.tt * BN + j;
+    if (t >= a.T) break;  // columns ascend: the rest are beyond T too
+    const uint32_t off = (uint32_t)(j * kRows + chl) * 4u;
+    uint4 v[kMaxClusterSplit];
+#pragma unroll
+    for (int z = 0; z < kMaxClusterSplit; ++z)
+      if (z < S) v[z] = ld_cluster_v4(src[z] + off);
+    uint32_t acc[4] = {v[0].x, v[0].y, v[0].z, v[0].w};
+#pragma unroll
+    for (int z = 1; z < kMaxClusterSplit; ++z) {
+      if (z < S) {
+        acc[0] = add_acc<DT>(acc[0], v[z].x);
+        acc[1] = add_acc<DT>(acc[1], v[z].y);
+        acc[2] = add_acc<DT>(acc[2], v[z].z);
+        acc[3] = add_acc<DT>(acc[3], v[z].w);
+      }
+    }
+    const size_t i0 = (size_t)t * a.n_out + ch;
+    if constexpr (EPI) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (ch + i < a.n_out) epi_one<DT>(a, EpiCh{sc[i], bi[i]}, i0 + i, acc[i]);
+    } else {
+      using OutT = decltype(convert_out<(OUT & 3)>(0u, 1.0f, false));
+      OutT o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = convert_out<(OUT & 3)>(acc[i], sc[i], has_scale);
+      OutT* yp = reinterpret_cast<OutT*>(a.Y) + i0;
+      if (vec) {
+        if constexpr (sizeof(OutT) == 4)
+          *reinterpret_cast<uint4*>(yp) = make_uint4(out_bits(o[0]), out_bits(o[1]), out_bits(o[2]), out_bits(o[3]));
+        else
+          *reinterpret_cast<uint2*>(yp) =
+              make_uint2(out_bits(o[0]) | (out_bits(o[1]) << 16), out_bits(o[2]) | (out_bits(o[3]) << 16));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (ch + i < a.n_out) yp[i] = o[i];
+      }
+    }
+  }
+}
+
 template <int DT, int IMG, int BN, int OUT, int XKB>
 __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
@@ -425,10 +503,28 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
   // Prologue done: the next kernel may start its own; global memory is touched
   // only after the previous kernel has completed (RAW/WAW order across launches).
   pdl_launch_dependents();
+  const UnitRange ur = my_units<XS>(a);
+  if (a.prefetch && warp == 0 && lane == 0 && ur.first < ur.end) {
+    // L2 hints for the first unit's operands while the previous kernel drains:
+    // a prefetch is not a memory access in the consistency model, so it may run
+    // ahead of the wait below (the copies that use the data come after it).
+    const Unit w0 = decode_unit(ur.first, a);
+    const int nkb = min(w0.kb1 - w0.kb0, C::STAGES);
+    if (nkb > 0) {
+      prefetch_l2(a.bpack + ((size_t)w0.ct * a.n_kb + w0.kb0) * C::CHUNK, (uint32_t)(nkb * C::CHUNK));
+      if constexpr (!XS && !C::GA) {
+        if (a.prefetch >= 2) {
+          for (int kb = w0.kb0; kb < w0.kb0 + nkb; ++kb) {  // boxes that start inside k only
+            prefetch_box_l2(&tmX, kb * C::KB, w0.tt * BN);
+            if (kb + 1 < a.n_kb) prefetch_box_l2(&tmX, kb * C::KB + C::KB / 2, w0.tt * BN);
+          }
+        }
+      }
+    }
+  }
   pdl_wait();
   const uint32_t tmem = tmem_base_sh;
   const uint64_t tmo = a.timeout_ns;
-  const UnitRange ur = my_units<XS>(a);
   uint8_t* const xregion = smem + (size_t)C::STAGES * C::STAGE;  // X-stationary mode only
 
   auto give_up = [&](int code) {
@@ -791,6 +887,24 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
             }
           }
         }
+      } else if (a.csplit) {
+        // on-chip split-K: park this split's partial tile in shared memory (the
+        // pipeline stages are idle: this CTA's only unit is fully accumulated);
+        // the cluster sums the partials after the role loops
+        if constexpr (!XS && !C::GA) {
+          uint32_t* xb = reinterpret_cast<uint32_t*>(smem);
+#pragma unroll 1
+          for (int c = 0; c < C::NCH; ++c) {
+            uint32_t r[C::CH];
+            tmem_ld_n<C::CH>(tbase + (uint32_t)(c * C::CH), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < C::CH; ++j) xb[(col0 + c * C::CH + j) * kRows + lq * 32 + lane] = r[j];
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acce_bar[acc]);
+        }
       } else {
         // split-K: publish this split's partial tile, the last arriving split reduces
         uint32_t* part = reinterpret_cast<uint32_t*>(a.ws);
@@ -851,6 +965,24 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
       }
     }
     if (lane == 0) bulk_wait<0>();  // this warp's tensor stores are complete before the CTA exits
+  }
+
+  if constexpr (!XS && !C::GA) {
+    static_assert(C::STAGES * C::STAGE >= BN * kRows * 4, "the stages hold a parked partial tile");
+    if (a.csplit) {
+      // Every thread of the cluster takes both barriers, whatever its role did
+      // (a bounded wait that gave up included): the first publishes the parked
+      // partials, the second keeps each CTA's shared memory alive until the
+      // whole cluster has read it.
+      __syncwarp();
+      cluster_arrive();
+      cluster_wait();
+      if (warp >= 2 && warp < 2 + C::EPI_WARPS)
+        csplit_reduce<DT, BN, OUT, C::EPI_WARPS>(a, decode_unit(ur.first, a), smem_u32(smem), warp - 2, lane);
+      __syncwarp();
+      cluster_arrive();
+      cluster_wait();
+    }
   }
 
   tc_fence_before();
@@ -1196,19 +1328,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
 
 // Launch with programmatic stream serialization, so the kernel's prologue can
 // overlap the tail of the previous kernel in the stream (see pdl_wait).
+// cluster > 1: launch as clusters of that many CTAs along x (grid a multiple of it).
 template <typename Kern>
 static cudaError_t launch_pdl(Kern kern, dim3 grid, int threads, int smem, cudaStream_t s, const CUtensorMap& tmX,
-                              const CUtensorMap& tmY, const CUtensorMap& tmW, const SpmmArgs& a) {
+                              const CUtensorMap& tmY, const CUtensorMap& tmW, const SpmmArgs& a, int cluster = 0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr.val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = &attr;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
   return cudaLaunchKernelEx(&cfg, kern, tmX, tmY, tmW, a);
 }
 
@@ -1234,7 +1374,9 @@ static cudaError_t launch_t(const CUtensorMap* tmX, const CUtensorMap* tmY, cons
   static std::atomic<uint64_t> opted{0};
   cudaError_t e = smem_opt_in(kern, C::SMEM, opted);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(p.grid), C::THREADS, C::SMEM, s, *tmX, *tmY, *tmW, a);
+  if (p.cluster && (XKB > 0 || IMG == IMG_GATHER || p.splits > kMaxClusterSplit || p.grid != p.units))
+    return cudaErrorInvalidValue;  // on-chip split-K: streaming kernel, one unit per CTA
+  return launch_pdl(kern, dim3(p.grid), C::THREADS, C::SMEM, s, *tmX, *tmY, *tmW, a, p.cluster ? p.splits : 0);
 }
 
 template <int DT, int IMG, int BN, int OUT>
@@ -1354,6 +1496,40 @@ static int max_clusters_t() {
     }
     cached = n > 0 ? n : -1;
     cache[dev].store(cached, std::memory_order_release);
+  }
+  return cached;
+}
+
+int stream_max_clusters(int size) {
+  static std::atomic<int> cache[64][kMaxClusterSplit + 1];
+  static std::atomic<uint64_t> opted{0};
+  int dev = 0;
+  if (size < 1 || size > kMaxClusterSplit) return -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  int cached = cache[dev][size].load(std::memory_order_acquire);
+  if (!cached) {
+    // every streaming configuration runs one CTA per SM, so one instance answers for all
+    using C = Cfg<DT_I8, IMG_SP24, 32, OUT_I32 | kOutDirect, 0>;
+    auto kern = spmm_kernel<DT_I8, IMG_SP24, 32, OUT_I32 | kOutDirect, 0>;
+    if (smem_opt_in(kern, C::SMEM, opted) != cudaSuccess) cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(size, 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = (unsigned)size;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cached = n > 0 ? n : -1;
+    cache[dev][size].store(cached, std::memory_order_release);
   }
   return cached;
 }

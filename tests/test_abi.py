@@ -70,6 +70,8 @@ def test_null_handle_paths():
     assert L.nm_query(None, None, None, None, None, None) == nm.NM_ERR_INVALID
     assert L.nm_device_status(None) == nm.NM_ERR_INVALID
     assert L.nm_export_sizes(None, None, None) == nm.NM_ERR_INVALID
+    assert L.nm_plan_query(None, 197, 0, None) == nm.NM_ERR_INVALID
+    assert L.nm_spmm_noalloc(None, None, 0, None, None, None) == nm.NM_ERR_INVALID
     L.nm_destroy(None)  # no-op
 
 

@@ -59,7 +59,8 @@ def _assert_float_close(Y_gpu: torch.Tensor, Y_ref: np.ndarray, dtype: str):
 @pytest.fixture(autouse=True)
 def _no_forced_plan(monkeypatch):
     for k in ("NMSPMM_FORCE_BN", "NMSPMM_FORCE_SPLITK", "NMSPMM_FORCE_XS", "NMSPMM_FORCE_GRID",
-              "NMSPMM_FORCE_PAIR", "NMSPMM_TMA_STORE"):
+              "NMSPMM_FORCE_PAIR", "NMSPMM_TMA_STORE", "NMSPMM_SPLIT_GLOBAL", "NMSPMM_CSPLIT",
+              "NMSPMM_PREFETCH"):
         monkeypatch.delenv(k, raising=False)
 
 
@@ -158,20 +159,111 @@ def test_spmm_fp16_scaled():
     _assert_float_close(Y, ref, "fp16")
 
 
+@pytest.mark.parametrize("mode", ["cluster", "global"])
 @pytest.mark.parametrize("bn", ["32", "64", "128", "192"])
 @pytest.mark.parametrize("split", ["1", "2", "3", "5"])
-def test_forced_tiles_and_splits_are_bit_identical(monkeypatch, bn, split):
-    """Adaptive parallelism must not change INT8 results at all."""
+def test_forced_tiles_and_splits_are_bit_identical(monkeypatch, bn, split, mode):
+    """Adaptive parallelism must not change INT8 results at all: every token
+    tile and split, with the partials reduced on chip (cluster) or in global
+    memory (workspace and arrival counters)."""
     W = _weights("int8", 200, 1280, seed=41)
     X = _acts("int8", 150, 1280, seed=42)
     s = inputs.scale_uniform(200, 0.001, 0.01, seed=43)
     ref = oracle.spmm(X.numpy(), W.numpy(), 2, 4, scale=s.numpy())
     monkeypatch.setenv("NMSPMM_FORCE_BN", bn)
     monkeypatch.setenv("NMSPMM_FORCE_SPLITK", split)
+    monkeypatch.setenv("NMSPMM_SPLIT_GLOBAL", "1" if mode == "global" else "0")
     h = nm.nm_compress(W.cuda(), 2, 4)
-    for _ in range(2):  # the second call reuses the re-armed split-K counters
+    plan = nm.nm_plan_query(h, 150, scaled=True)
+    assert plan["splits"] == int(split) and plan["bn"] == int(bn)
+    assert plan["cluster"] == (1 if (mode == "cluster" and split != "1") else 0)
+    for _ in range(2):  # the second call reuses the workspace and its counters
         Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
         assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("S", [2, 3, 4, 8])
+@pytest.mark.parametrize("bn", ["32", "64", "128"])
+@pytest.mark.parametrize("n_out", [200, 198])
+@pytest.mark.parametrize("N,M", [(2, 4), (4, 8)])
+def test_cluster_split_int8_outputs_bit_exact(monkeypatch, S, bn, n_out, N, M):
+    """On-chip split-K: int32 and scaled fp32 outputs, whole (n_out % 4 == 0,
+    16-byte stores) and ragged (element stores) channel groups, ragged T."""
+    K, T = 2048, 197
+    W = _weights("int8", n_out, K, seed=401 + n_out)
+    X = _acts("int8", T, K, seed=402)
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=403)
+    monkeypatch.setenv("NMSPMM_FORCE_BN", bn)
+    monkeypatch.setenv("NMSPMM_FORCE_SPLITK", str(S))
+    h = nm.nm_compress(W.cuda(), N, M)
+    assert nm.nm_plan_query(h, T)["cluster"] == 1
+    for scaled in (False, True):
+        Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda() if scaled else None)
+        torch.cuda.synchronize()
+        assert nm.nm_device_status(h) == nm.NM_OK
+        ref = oracle.spmm(X.numpy(), W.numpy(), N, M, scale=s.numpy() if scaled else None)
+        assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("S", [2, 4, 8])
+@pytest.mark.parametrize("n_out", [256, 190])
+def test_cluster_split_float_within_tolerance(monkeypatch, dtype, S, n_out):
+    K, T = 2048, 77
+    W = _weights(dtype, n_out, K, seed=411)
+    X = _acts(dtype, T, K, seed=412)
+    monkeypatch.setenv("NMSPMM_FORCE_SPLITK", str(S))
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    assert nm.nm_plan_query(h, T)["cluster"] == 1
+    Y = nm.nm_spmm(h, X.cuda())
+    torch.cuda.synchronize()
+    assert nm.nm_device_status(h) == nm.NM_OK
+    _assert_float_close(Y, oracle.spmm(_np(X, dtype), _np(W, dtype), 2, 4, dtype=dtype), dtype)
+
+
+def test_cluster_split_runtime_output_stage_bit_exact(monkeypatch):
+    """nm_spmm_ex under the on-chip split: scale, bias and int8 requantisation."""
+    K, T, n_out = 3072, 197, 198
+    W = _weights("int8", n_out, K, seed=421)
+    X = _acts("int8", T, K, seed=422)
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=423)
+    b = inputs.scale_uniform(n_out, -2.0, 2.0, seed=424)
+    monkeypatch.setenv("NMSPMM_FORCE_SPLITK", "6")
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    assert nm.nm_plan_query(h, T, scaled=True)["cluster"] == 1
+    for out in ("int8", "float32"):
+        Y = nm.nm_spmm_ex(h, X.cuda(), scale=s.cuda(), bias=b.cuda(), out=out, out_scale=0.05)
+        torch.cuda.synchronize()
+        ref = oracle.spmm_epilogue(X.numpy(), W.numpy(), 2, 4, scale=s.numpy(), bias=b.numpy(), out=out,
+                                   out_scale=0.05)
+        assert np.array_equal(Y.cpu().numpy(), ref["exact"]), out
+
+
+@pytest.mark.parametrize("N,M", [(2, 4), (4, 8)])
+@pytest.mark.parametrize("n_out,K", [(768, 768), (2304, 768), (3072, 768), (768, 3072)])
+def test_planner_splits_small_token_counts_on_chip(n_out, K, N, M):
+    """At a few tokens the unsplit tiles of the long-k ViT-B layer (fc2, 12
+    k-blocks on 6 to 12 CTAs) leave almost every SM idle: the planner splits k
+    over a cluster.  The 3-k-block layers are not split (the on-chip reduction
+    costs more than their k loop), and at T = 12608 nothing is split.  Whatever
+    the plan, the result is the oracle's."""
+    W = _weights("int8", n_out, K, seed=431)
+    h = nm.nm_compress(W.cuda(), N, M)
+    big = nm.nm_plan_query(h, 12608, scaled=True)
+    assert big["splits"] == 1 and big["cluster"] == 0
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=433)
+    for T in (16, 64, 197):
+        small = nm.nm_plan_query(h, T, scaled=True)
+        if K == 3072 and T <= 64:
+            assert small["splits"] > 1 and small["cluster"] == 1, (T, small)
+        if K == 768:
+            assert small["splits"] == 1, (T, small)
+        if small["splits"] > 1:
+            assert small["cluster"] == 1 and small["grid"] == small["units"]
+        X = _acts("int8", T, K, seed=432 + T)
+        Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
+        ref = oracle.spmm(X.numpy(), W.numpy(), N, M, scale=s.numpy())
+        assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32)), T
 
 
 @pytest.mark.parametrize("grid", ["5", "148"])
@@ -246,11 +338,13 @@ def test_streaming_mode_many_units_per_cta(monkeypatch, grid):
     assert np.array_equal(Y.cpu().numpy(), oracle.spmm(X.numpy(), W.numpy(), 2, 4))
 
 
+@pytest.mark.parametrize("mode", ["cluster", "global"])
 @pytest.mark.parametrize("split", ["1", "4"])
-def test_forced_split_fp16_within_tolerance(monkeypatch, split):
+def test_forced_split_fp16_within_tolerance(monkeypatch, split, mode):
     W = _weights("fp16", 256, 2048, seed=51)
     X = _acts("fp16", 40, 2048, seed=52)
     monkeypatch.setenv("NMSPMM_FORCE_SPLITK", split)
+    monkeypatch.setenv("NMSPMM_SPLIT_GLOBAL", "1" if mode == "global" else "0")
     h = nm.nm_compress(W.cuda(), 2, 8)
     Y = nm.nm_spmm(h, X.cuda())
     _assert_float_close(Y, oracle.spmm(_np(X, "fp16"), _np(W, "fp16"), 2, 8, dtype="fp16"), "fp16")
@@ -271,10 +365,20 @@ def test_forced_tile_float_within_tolerance(monkeypatch, dtype, bn):
 # --------------------------------------------------------------------------- full-size workloads (sampled)
 
 
-def _sampled_rows(T, count, seed):
+def _sampled_rows(T, count, seed, h=None, scaled=False):
+    """Random rows plus, when the handle is given, the first and last token of
+    every token tile of the plan the call uses (every half tile for the two-SM
+    kernel, whose CTAs each hold half of the tile's tokens), so that every
+    (channel tile, token tile) pair the kernel writes is compared: all
+    columns of each row are checked."""
     rng = np.random.default_rng(seed)
     rows = set(rng.choice(T, size=min(count, T), replace=False).tolist())
     rows.update({0, T - 1})
+    if h is not None:
+        plan = nm.nm_plan_query(h, T, scaled=scaled)
+        step = plan["bn"] // 2 if plan["pair"] else plan["bn"]
+        for t0 in range(0, T, step):
+            rows.update({t0, min(t0 + step, T) - 1})
     return np.array(sorted(rows))
 
 
@@ -291,7 +395,7 @@ def test_vit_b_int8_sampled_rows(layer):
     W, X, s = layer.weight(), layer.activation(), layer.scale()
     h = nm.nm_compress(W.cuda(), layer.N, layer.M)
     Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
-    rows = _sampled_rows(layer.T, 48, layer.seed)
+    rows = _sampled_rows(layer.T, 48, layer.seed, h, scaled=True)
     ref = oracle.spmm(X.numpy()[rows], W.numpy(), layer.N, layer.M, scale=s.numpy())
     assert np.array_equal(Y.cpu().numpy()[rows].view(np.uint32), ref.view(np.uint32))
 
@@ -301,7 +405,7 @@ def test_vit_l_fp16_sampled_rows(layer):
     W, X = layer.weight(), layer.activation()
     h = nm.nm_compress(W.cuda(), layer.N, layer.M)
     Y = nm.nm_spmm(h, X.cuda())
-    rows = _sampled_rows(layer.T, 32, layer.seed)
+    rows = _sampled_rows(layer.T, 32, layer.seed, h)
     ref = oracle.spmm(_np(X, "fp16")[rows], _np(W, "fp16"), layer.N, layer.M, dtype="fp16")
     _assert_float_close(Y[rows.tolist()], ref, "fp16")
 
@@ -311,7 +415,7 @@ def test_swin_t_int8_sampled_rows(layer):
     W, X, s = layer.weight(), layer.activation(), layer.scale()
     h = nm.nm_compress(W.cuda(), layer.N, layer.M)
     Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
-    rows = _sampled_rows(layer.T, 48, layer.seed)
+    rows = _sampled_rows(layer.T, 48, layer.seed, h, scaled=True)
     ref = oracle.spmm(X.numpy()[rows], W.numpy(), layer.N, layer.M, scale=s.numpy())
     assert np.array_equal(Y.cpu().numpy()[rows].view(np.uint32), ref.view(np.uint32))
 
@@ -327,7 +431,7 @@ def test_vit_b_mixed_sequence(T):
         outs.append((l, X, W, s, h, nm.nm_spmm(h, X.cuda(), scale=s.cuda())))
     torch.cuda.synchronize()
     for l, X, W, s, h, Y in outs:
-        rows = _sampled_rows(l.T, 16, l.seed) if T > 1000 else np.arange(T)
+        rows = _sampled_rows(l.T, 16, l.seed, h, scaled=True) if T > 1000 else np.arange(T)
         ref = oracle.spmm(X.numpy()[rows], W.numpy(), l.N, l.M, scale=s.numpy())
         assert np.array_equal(Y.cpu().numpy()[rows].view(np.uint32), ref.view(np.uint32)), l.name
 

@@ -3,12 +3,15 @@
 nm_spmm_noalloc serves callers that cannot allocate device memory (a serving
 engine that owns nearly all of HBM through its own pool; latency-critical code
 that must not call cudaMalloc/cudaFree, which can synchronise the device).  Its
-split-K scratch is a fixed array inside the library instead of a workspace the
-handle allocates.  These tests force shapes onto the split-K path so the array
-is really used, run two calls in a row (the array keeps the previous call's
-contents), and compare every output with the existing entry point: bit-exact
-for INT8, the FP16 tolerance of the parity suite for FP16.  This file is
-collected last so a failure here cannot hide the other suites' results.
+scratch for a global-memory split-K is a fixed array inside the library instead
+of a workspace the handle allocates.  The planner's own plans never need it
+(they do not split k, or they reduce the splits on chip), so these tests force
+shapes onto the global-memory split-K path so the array is really used, run two
+calls in a row (the array keeps the previous call's contents), and compare
+every output with the existing entry point: bit-exact for INT8, the FP16
+tolerance of the parity suite for FP16.  One test runs the default plans,
+which must match nm_spmm as well.  This file is collected last so a failure
+here cannot hide the other suites' results.
 """
 import ctypes
 
@@ -32,6 +35,7 @@ def _call_noalloc(h, X, Y, scale):
 @pytest.mark.parametrize("N,M,scaled", [(2, 4, True), (1, 4, False), (4, 8, True)])
 def test_noalloc_int8_matches_nm_spmm_twice(monkeypatch, split, N, M, scaled):
     monkeypatch.setenv("NMSPMM_FORCE_SPLITK", split)
+    monkeypatch.setenv("NMSPMM_SPLIT_GLOBAL", "1")
     W = inputs.int8_uniform((768, 768), -127, 127, seed=71).cuda()
     s = inputs.scale_uniform(768, 0.001, 0.01, seed=73).cuda() if scaled else None
     h = nm.nm_compress(W, N, M)
@@ -48,6 +52,7 @@ def test_noalloc_int8_matches_nm_spmm_twice(monkeypatch, split, N, M, scaled):
 
 def test_noalloc_fp16_within_tolerance_twice(monkeypatch):
     monkeypatch.setenv("NMSPMM_FORCE_SPLITK", "4")
+    monkeypatch.setenv("NMSPMM_SPLIT_GLOBAL", "1")
     W = inputs.float_normal((256, 2048), 0.02, seed=81, dtype="fp16").cuda()
     h = nm.nm_compress(W, 2, 4)
     for call in range(2):
@@ -61,9 +66,28 @@ def test_noalloc_fp16_within_tolerance_twice(monkeypatch):
         assert torch.linalg.norm(got.double() - want).item() <= 1e-3 * torch.linalg.norm(want).item()
 
 
+@pytest.mark.parametrize("T", [197, 12608])
+@pytest.mark.parametrize("n_out,K", [(768, 768), (768, 3072)])
+def test_noalloc_default_plan_matches_nm_spmm_twice(monkeypatch, T, n_out, K):
+    for k in ("NMSPMM_FORCE_SPLITK", "NMSPMM_SPLIT_GLOBAL", "NMSPMM_FORCE_BN"):
+        monkeypatch.delenv(k, raising=False)
+    W = inputs.int8_uniform((n_out, K), -127, 127, seed=75).cuda()
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=76).cuda()
+    h = nm.nm_compress(W, 2, 4)
+    for call in range(2):
+        X = inputs.int8_uniform((T, K), -128, 127, seed=77 + call).cuda()
+        want = nm.nm_spmm(h, X, scale=s)
+        got = torch.full_like(want, -1)
+        assert _call_noalloc(h, X, got, s) == nm.NM_OK, nm.nm_last_error()
+        torch.cuda.synchronize()
+        assert nm.nm_device_status(h) == nm.NM_OK
+        assert torch.equal(got.view(torch.int32), want.view(torch.int32)), f"call {call}"
+
+
 def test_noalloc_rejects_scratch_beyond_the_limit(monkeypatch):
     monkeypatch.setenv("NMSPMM_FORCE_BN", "128")
     monkeypatch.setenv("NMSPMM_FORCE_SPLITK", "3")
+    monkeypatch.setenv("NMSPMM_SPLIT_GLOBAL", "1")
     W = inputs.int8_uniform((512, 768), -127, 127, seed=91).cuda()
     X = inputs.int8_uniform((1024, 768), -128, 127, seed=92).cuda()
     h = nm.nm_compress(W, 2, 4)
