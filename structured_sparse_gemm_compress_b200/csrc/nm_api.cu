@@ -555,7 +555,7 @@ nm_status spmm_impl(const nm_handle* hc, const void* X, int64_t T, void* Y, cons
   // timeline builds only: device buffer of grid * kTraceStride int64 given as an integer address
   if (const char* tp = getenv("NMSPMM_TRACE_PTR")) a.trace = reinterpret_cast<long long*>(strtoull(tp, nullptr, 0));
 #endif
-  a.prefetch = std::max(0, std::min(2, env_int("NMSPMM_PREFETCH", 1)));
+  a.prefetch = std::max(0, std::min(2, env_int("NMSPMM_PREFETCH", 2)));
   if (p.cluster) {
     a.csplit = 1;  // partials summed on chip: no workspace
   } else if (p.splits > 1) {

@@ -87,6 +87,35 @@ def test_int8_output_stage_bit_exact(N, M, out, scaled, biased):
         assert (q == 127).any() and (q == -128).any() and ((q > -128) & (q < 127)).mean() > 0.3
 
 
+@pytest.mark.parametrize("out,os_", [("float32", 1.0), ("int8", 2.0 ** -24), ("int8", 2.0 ** -21)])
+def test_output_stage_conversions_at_extreme_accumulators(out, os_):
+    """The runtime stage's int32 -> fp32 conversion (rounded to nearest even)
+    and int8 rounding across the whole accumulator range: k = 2^17, rows of
+    all +127 / all -127 / random signs against X of -128 or random values, so
+    |acc| spans the exact range below 2^24, the rounded range above it, and
+    reaches 128 * 127 * 2^17 (just under 2^31).  Scale 1 and a zero bias keep
+    the value the conversion itself; bit-exact against the oracle."""
+    n_out, K, T = 128, 1 << 17, 33
+    sign = torch.where(inputs.int8_uniform((n_out, K), 0, 1, seed=91) > 0, 127, -127).to(torch.int8)
+    sign[:8] = 127
+    sign[8:16] = -127
+    for r in range(16, n_out):  # a run of equal signs of growing length: |acc| from 2^20 to 2^27
+        sign[r, : 64 * r] = 127 if r % 2 else -127
+    X = inputs.int8_uniform((T, K), -128, 127, seed=92)
+    X[:8] = -128
+    h = nm.nm_compress(sign.cuda(), 4, 4)
+    one = torch.ones(n_out, dtype=torch.float32)
+    zero = torch.zeros(n_out, dtype=torch.float32)
+    Y = nm.nm_spmm_ex(h, X.cuda(), scale=one.cuda(), bias=zero.cuda(), out=out, out_scale=os_)
+    torch.cuda.synchronize()
+    acc = oracle.gemm(X.numpy(), sign.numpy())
+    assert np.abs(acc.astype(np.int64)).max() == 128 * 127 * K
+    mag = np.abs(acc.astype(np.int64))
+    assert (mag > 2 ** 24).mean() > 0.2 and (mag < 2 ** 22).mean() > 0.2
+    ref = oracle.epilogue(acc, one.numpy(), zero.numpy(), "none", out, os_)
+    assert np.array_equal(_gpu_np(Y), ref["exact"])
+
+
 def _gelu_tol(v: np.ndarray, g: np.ndarray) -> np.ndarray:
     return 4e-7 * np.abs(v) + 2e-6 * np.abs(g) + 1e-30
 
