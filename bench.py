@@ -103,6 +103,9 @@ class ClockSampler:
     def mark_end(self):
         self.t1 = time.time()
 
+    def poke(self):
+        pass
+
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
@@ -199,22 +202,29 @@ class NvmlSampler:
         self._thread.start()
         return self
 
-    def _poll(self):
+    def _sample(self):
         n = self._nvml
         get_reasons = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
             n.nvmlDeviceGetCurrentClocksThrottleReasons
+        try:
+            sm = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+            rs = get_reasons(self._h)
+            pw = n.nvmlDeviceGetPowerUsage(self._h) / 1000.0 if len(self.samples) % 8 == 0 else None
+            self.samples.append((sm, rs, pw))
+        except Exception:
+            pass
+
+    def _poll(self):
         while self._run:
             if self._inside:
-                try:
-                    sm = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
-                    rs = get_reasons(self._h)
-                    pw = n.nvmlDeviceGetPowerUsage(self._h) / 1000.0
-                    self.samples.append((sm, rs, pw))
-                except Exception:
-                    pass
-                time.sleep(0.0005)
+                self._sample()
             else:
                 time.sleep(0.0002)
+
+    def poke(self):
+        """One sample taken now (call while the GPU is busy inside the region)."""
+        if self._nvml is not None and self._inside:
+            self._sample()
 
     def mark_start(self):
         if self._fallback is not None:
@@ -225,6 +235,8 @@ class NvmlSampler:
         if self._fallback is not None:
             return self._fallback.mark_end()
         self._inside = False
+
+
 
     def __exit__(self, *exc):
         if self._fallback is not None:
@@ -241,8 +253,9 @@ class NvmlSampler:
                     "samples": 0, "samples_in_timed_region": 0, "source": "nvml"}
         sm = [x[0] for x in self.samples]
         reasons = sorted({name for _, rs, _ in self.samples for name, bit in self.REASONS if rs & bit})
+        pw = [x[2] for x in self.samples if x[2] is not None]
         return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "power_w_max": round(max(x[2] for x in self.samples), 1),
+                "reasons": reasons, "power_w_max": round(max(pw), 1) if pw else None,
                 "samples": len(sm), "samples_in_timed_region": len(sm), "source": "nvml, ~1 ms polling"}
 
 
@@ -887,10 +900,12 @@ def main() -> None:
         if graphs:
             for g in graphs:
                 g.replay()
+                clk.poke()
         else:
             for k in range(args.steps):
                 step()
         stop.record(stream)
+        clk.poke()
         torch.cuda.synchronize()
         clk.mark_end()
         barrier()

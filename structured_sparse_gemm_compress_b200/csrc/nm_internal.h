@@ -120,7 +120,10 @@ struct SpmmArgs {
 // Timeline trace layout (builds with NM_TRACE): per CTA kTraceStride int64
 // slots: [kind][index], kinds below, kTraceMax indices each.
 constexpr int kTraceMax = 64;
-enum : int { TR_P_ISSUE = 0, TR_M_FULL, TR_M_DONE, TR_M_ACCE, TR_E_START, TR_E_END, TR_KINDS };
+// TR_GT holds %globaltimer (ns, comparable across SMs) at kernel entry (0),
+// after the wait on the previous kernel (1), after the role loops (2) and at
+// exit (3), written by thread 0.
+enum : int { TR_P_ISSUE = 0, TR_M_FULL, TR_M_DONE, TR_M_ACCE, TR_E_START, TR_E_END, TR_GT, TR_KINDS };
 constexpr int kTraceStride = TR_KINDS * kTraceMax;
 
 cudaError_t launch_compress(const nm_handle* h, const void* W, cudaStream_t s);

@@ -148,9 +148,17 @@ __host__ __device__ constexpr uint32_t make_idesc() {
       a.trace[(size_t)blockIdx.x * kTraceStride + (kind) * kTraceMax + (idx)] =            \
           (long long)clock64();                                                            \
   } while (0)
+#define NM_TG(idx)                                                                                   \
+  do {                                                                                               \
+    if (a.trace && threadIdx.x == 0)                                                                 \
+      a.trace[(size_t)blockIdx.x * kTraceStride + TR_GT * kTraceMax + (idx)] = (long long)globaltimer(); \
+  } while (0)
 #else
 #define NM_TR(kind, idx) \
   do {                   \
+  } while (0)
+#define NM_TG(idx) \
+  do {             \
   } while (0)
 #endif
 
@@ -470,6 +478,7 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  NM_TG(0);
 
   if (threadIdx.x == 0) {
     // gather image with gather warps: the producer's arrive plus one per gather warp
@@ -523,6 +532,7 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
     }
   }
   pdl_wait();
+  NM_TG(1);
   const uint32_t tmem = tmem_base_sh;
   const uint64_t tmo = a.timeout_ns;
   uint8_t* const xregion = smem + (size_t)C::STAGES * C::STAGE;  // X-stationary mode only
@@ -967,6 +977,7 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
     if (lane == 0) bulk_wait<0>();  // this warp's tensor stores are complete before the CTA exits
   }
 
+  NM_TG(2);
   if constexpr (!XS && !C::GA) {
     static_assert(C::STAGES * C::STAGE >= BN * kRows * 4, "the stages hold a parked partial tile");
     if (a.csplit) {
@@ -991,6 +1002,7 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  NM_TG(3);
 }
 
 // ------------------------------------------------------------------ CTA-pair kernel
@@ -1060,6 +1072,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
+  NM_TG(0);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
@@ -1088,6 +1101,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
   tc_fence_after();
   pdl_launch_dependents();
   pdl_wait();
+  NM_TG(1);
   const uint32_t tmem = tmem_base_sh;
   const uint64_t tmo = a.timeout_ns;
   const uint32_t full_lead0 = mapa_shared(smem_u32(&full_bar[0]), 0);  // leader's stage barriers
@@ -1315,6 +1329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
 
   // Teardown: every remote arrive and copy of the pair is done before either
   // CTA frees tensor memory or exits.
+  NM_TG(2);
   tc_fence_before();
   __syncthreads();
   cluster_sync();
@@ -1322,6 +1337,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
     tc_fence_after();
     tmem_dealloc_cg<2>(tmem, C::TMEM_COLS);
   }
+  NM_TG(3);
 }
 
 // ------------------------------------------------------------------ host launch

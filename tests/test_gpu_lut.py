@@ -19,12 +19,16 @@ def test_lut_predicts_held_out_sequences():
               lut.measure_sequence(layers, lut.random_assignment(len(layers), 10 + i), T, reps=3, ws=ws))
              for T in Ts for i in range(3)]
     L.calibrate(calib)
+    errs = []
     for T in Ts:
         for i in range(3):
             asg = lut.random_assignment(len(layers), 50 + i)
             meas = lut.measure_sequence(layers, asg, T, reps=3, ws=ws)
             pred = L.predict(layers, asg, T)
-            assert abs(pred - meas) <= 0.2 * meas, (T, asg, pred, meas)
+            errs.append(abs(pred - meas) / meas)
+            # a latency budget enforced through the predictor is only as good as this bound
+            assert errs[-1] <= 0.10, (T, asg, pred, meas)
+    assert sum(errs) / len(errs) <= 0.05, errs
     # the profiled table answers any T through interpolation
     assert L.lookup(768, 2304, "2:4", 2000) > 0
 
@@ -46,7 +50,7 @@ def test_lut_with_tile_shared_patterns():
     for i in range(3):
         asg = lut.random_assignment(len(layers), 90 + i, tuple(pats))
         meas = lut.measure_sequence(layers, asg, 2048, reps=3, ws=ws)
-        assert abs(L.predict(layers, asg, 2048) - meas) <= 0.2 * meas, (asg, meas)
+        assert abs(L.predict(layers, asg, 2048) - meas) <= 0.10 * meas, (asg, meas)
 
 
 def test_tile_shared_keeps_at_most_the_per_row_mass():
