@@ -221,6 +221,28 @@ def test_cluster_split_float_within_tolerance(monkeypatch, dtype, S, n_out):
     _assert_float_close(Y, oracle.spmm(_np(X, dtype), _np(W, dtype), 2, 4, dtype=dtype), dtype)
 
 
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_cluster_split_runtime_output_stage_float(monkeypatch, dtype):
+    """nm_spmm_ex on an FP16/BF16 handle under the on-chip split: scale, bias
+    and GELU, fp32 output, within the float tolerance of the fp64 oracle."""
+    K, T, n_out = 2048, 61, 190
+    W = _weights(dtype, n_out, K, seed=441)
+    X = _acts(dtype, T, K, seed=442)
+    s = inputs.scale_uniform(n_out, 0.5, 2.0, seed=443)
+    b = inputs.scale_uniform(n_out, -1.0, 1.0, seed=444)
+    monkeypatch.setenv("NMSPMM_FORCE_SPLITK", "4")
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    assert nm.nm_plan_query(h, T, scaled=True)["cluster"] == 1
+    Y = nm.nm_spmm_ex(h, X.cuda(), scale=s.cuda(), bias=b.cuda(), act="gelu", out="float32")
+    torch.cuda.synchronize()
+    ref = oracle.spmm_epilogue(_np(X, dtype), _np(W, dtype), 2, 4, scale=s.numpy(), bias=b.numpy(), act="gelu",
+                               out="float32", dtype=dtype)["pre"]
+    got = Y.double().cpu().numpy()
+    amax, frob = TOL[dtype]
+    assert np.abs(got - ref).max() <= amax * np.abs(ref).max()
+    assert np.linalg.norm(got - ref) <= frob * np.linalg.norm(ref)
+
+
 def test_cluster_split_runtime_output_stage_bit_exact(monkeypatch):
     """nm_spmm_ex under the on-chip split: scale, bias and int8 requantisation."""
     K, T, n_out = 3072, 197, 198
