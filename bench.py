@@ -362,6 +362,7 @@ def roofline_point(l, us: float, pk: dict, out_es: int | None = None, biased: bo
     t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9) * 1e6
     t_roof = max(t_tc, t_hbm)
     return {"us": round(us, 2), "dense_eq_tops": round(ops / us / 1e6, 1),
+            "useful_tops": round(l.kept_ops() / us / 1e6, 1),
             "bound": "tensor" if t_tc > t_hbm else "hbm", "roofline_us": round(t_roof, 2),
             "frac": round(t_roof / us, 3)}
 
@@ -557,7 +558,15 @@ def run_cosearch(args) -> None:
     print(json.dumps(line), flush=True)
 
 
-def _graph_us(launch, stream, reps: int = 20, replays: int = 5) -> float:
+def _graph_stats(launch, stream, reps: int = 20, replays: int = 11) -> tuple[float, float, float]:
+    """(median, p10, p90) in us of one launch over `replays` replays of a CUDA
+    graph of `reps` back-to-back launches (see _graph_us)."""
+    ts = _graph_us(launch, stream, reps, replays, all_replays=True)
+    q = np.percentile(ts, [50, 10, 90])
+    return float(q[0]), float(q[1]), float(q[2])
+
+
+def _graph_us(launch, stream, reps: int = 20, replays: int = 5, all_replays: bool = False):
     """Time (us) of one launch: `reps` launches back to back in one CUDA graph,
     events around each replay, median over `replays` replays.  Our kernels and
     cuBLAS's are timed by this same function, so launch overlap (programmatic
@@ -583,7 +592,7 @@ def _graph_us(launch, stream, reps: int = 20, replays: int = 5) -> float:
         torch.cuda.synchronize()
         ts.append(a.elapsed_time(b) * 1e3 / reps)
     del g
-    return statistics.median(ts)
+    return ts if all_replays else statistics.median(ts)
 
 
 def measure_int8_peak(device) -> dict:
@@ -755,6 +764,7 @@ def measure_config(name: str, args, pk: dict, min_region_ms: float = 200.0, devi
     tot_roof = sum(p["roofline_us"] for p in per)
     line = {"config": {"workload": desc}, "metric": "dense-equivalent TOPS over the sequence", "unit": "TOPS",
             "value": total_ops / (seq_ms * 1e-3) / 1e12, "sequence_us": round(seq_ms * 1e3, 2),
+            "useful_tops": sum(l.kept_ops() for l in ls) / (seq_ms * 1e-3) / 1e12,
             "sum_of_kernel_us": round(sum(p["us"] for p in per), 2),
             "per_problem_note": ("us: that launch alone, 20 back to back in a CUDA graph (median of 5 replays); "
                                  "cuBLAS timed the same way"),
@@ -917,6 +927,7 @@ def main() -> None:
 
     ops_step = sum(l.dense_ops() for l in ls)
     value = whole_job_tops(ops_step, args.steps, world, ms)
+    useful = whole_job_tops(sum(l.kept_ops() for l in ls), args.steps, world, ms)
 
     # Roofline of the dominant kernel (the SpMM).  Its average launch duration is
     # the main stream's timed region (start/stop events on that stream) over the
@@ -947,9 +958,10 @@ def main() -> None:
             cublas[name] = _graph_us(lambda st, Xd=Xd, Wt=Wt: torch._int_mm(Xd, Wt), stream)
         for i, l in enumerate(ls):
             d = devb[l.name]
-            us = _graph_us(lambda st, i=i, d=d: nm.nm_spmm(handles[i], d["X"], Y=Ys[i], scale=d["s"], stream=st),
-                           stream)
+            us, p10, p90 = _graph_stats(
+                lambda st, i=i, d=d: nm.nm_spmm(handles[i], d["X"], Y=Ys[i], scale=d["s"], stream=st), stream)
             rp = roofline_point(l, us, pk)
+            rp["us_p10"], rp["us_p90"] = round(p10, 2), round(p90, 2)
             rp["hbm_frac"] = round(alg_bytes(l) / (us * 1e-6) / 1e9 / pk["hbm_gbs"], 3)
             rp["cublas_int8_dense_us"] = round(cublas[l.name], 2)
             rp["vs_cublas"] = round(cublas[l.name] / us, 3)
@@ -1007,6 +1019,15 @@ def main() -> None:
         cpu = {"value": ops / secs / 1e12, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
                "sample": f"first {rows} of 12608 tokens of each of the 16 (layer, N:M) problems "
                          f"(compress + decompress + triple-loop GEMM), {secs:.1f} s"}
+        # the same oracle on one core, on an eighth of the sample
+        all_threads = oracle.threads()
+        oracle.set_threads(1)
+        try:
+            s1, o1 = cpu_oracle_run(ls, max(16, rows // 8))
+        finally:
+            oracle.set_threads(all_threads)
+        cpu["one_core"] = {"value": o1 / s1 / 1e12, "unit": UNIT, "cores": 1,
+                           "sample": f"first {max(16, rows // 8)} tokens of each problem, {s1:.1f} s"}
 
     del graphs, built
     if dist is not None:
@@ -1030,13 +1051,16 @@ def main() -> None:
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk.summary(),
+        "useful_tops": useful,
         "spmm_launch_us_avg": 1e3 * ms_local / (args.steps * len(ls)),
         "pack_us_per_step": pack_us,
         "pack_overlapped": True,
         "int8_dense_peak_tops_measured": None if int8_peak is None else round(int8_peak["int8_dense_tops"], 1),
         "per_layer_note": ("each problem alone and cuBLAS's int8 GEMM of the same shape, both as 20 back-to-back "
-                           "launches in a CUDA graph (median of 5 replays); hbm_frac = algorithmic bytes / time / "
-                           "measured HBM; frac = roofline (max of HBM and tensor time, INT8 peak measured) / time"),
+                           "launches in a CUDA graph (ours: median and p10/p90 of 11 replays; cuBLAS: median of 5); "
+                           "hbm_frac = algorithmic bytes / time / measured HBM; frac = roofline (max of HBM and "
+                           "tensor time, INT8 peak measured) / time; useful_tops counts the kept weights only "
+                           "((N/M) x dense-equivalent)"),
         "per_layer": per_layer,
         "cublas_int8_dense": cublas,
     }

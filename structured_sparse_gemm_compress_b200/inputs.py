@@ -85,6 +85,10 @@ class Layer:
         """Dense-equivalent operation count 2*T*K*n_out."""
         return 2 * self.T * self.K * self.n_out
 
+    def kept_ops(self) -> int:
+        """Useful operations: 2 per kept weight and token, (N/M) x the dense-equivalent count."""
+        return 2 * self.T * (self.K // self.M) * self.N * self.n_out
+
 
 def _vit_block(d: int, hidden: int):
     return [("qkv", d, 3 * d), ("proj", d, d), ("fc1", d, hidden), ("fc2", hidden, d)]
