@@ -73,7 +73,7 @@ def _stage_stats(tr: np.ndarray, pair: bool) -> dict:
             "epilogue_cycles_per_tile": med(epi), "tile_period_cycles": med(period)}
 
 
-def run(problems: list[str], sequence_reps: int = 1) -> dict:
+def run(problems: list[str], raw_out: bool = False) -> dict:
     build.build(trace=True)
     import structured_sparse_gemm_compress_b200 as nm
     if nm._lib is not None:
@@ -105,11 +105,16 @@ def run(problems: list[str], sequence_reps: int = 1) -> dict:
         gt = tr[:, GT, :4]
         gt = gt[gt[:, 0] > 0]
         base = gt[:, 0].min() if base is None else base
+        raw = {f"cta{b}": {k: [int(x) for x in tr[b, i, :24]] for i, k in
+                           enumerate(("p_issue", "m_full", "m_done", "m_acce", "e_start", "e_end"))}
+               for b in (0, 1) if b < tr.shape[0]}
         r = {"problem": p["name"], "plan": p["plan"], **_stage_stats(tr, bool(p["plan"]["pair"])),
              "entry_us": round((gt[:, 0].min() - base) / 1e3, 2), "first_wait_return_us": round((gt[:, 1].min() - base) / 1e3, 2),
              "exit_first_us": round((gt[:, 3].min() - base) / 1e3, 2), "exit_last_us": round((gt[:, 3].max() - base) / 1e3, 2)}
         if prev_exit is not None:
             r["prev_last_exit_to_first_wait_return_us"] = round((gt[:, 1].min() - prev_exit) / 1e3, 2)
+        if raw_out:
+            r["raw_first_ctas"] = raw
         prev_exit = gt[:, 3].max()
         out.append(r)
         p["h"].destroy()
@@ -121,10 +126,11 @@ def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--problems", required=True, help="comma-separated, e.g. vitb.qkv/2:4,vitb.fc2/2:4")
     ap.add_argument("--out", default=None)
+    ap.add_argument("--raw", action="store_true", help="also keep the first CTAs' raw stamps (first 24 of each kind)")
     a = ap.parse_args()
-    res = run(a.problems.split(","))
+    res = run(a.problems.split(","), raw_out=a.raw)
     for r in res["problems"]:
-        print(json.dumps(r))
+        print(json.dumps({k: v for k, v in r.items() if k != "raw_first_ctas"}))
     if a.out:
         json.dump(res, open(a.out, "w"), indent=1)
 
