@@ -293,9 +293,18 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
   // CTA-pair mode (M = 256 per MMA, one issuing thread per two SMs): whenever
   // there are enough 256-channel x BN-token tiles to occupy every resident pair.
   const int forced_pair = env_int("NMSPMM_FORCE_PAIR", -1);  // -1 auto, 0 off, 1 on
-  // Measured on B200: the pair pays off once the k loop is long (>= 2 KB of X per token), where
-  // per-stage issue cost and X re-reads dominate; shorter k stays on one CTA.
-  const bool pair_default = h->k * nm::elem_bytes(h->dt) >= 2048;  // >= 2 KB of X per token
+  // Measured on B200 (CUDA-graph timing of both kernels, INT8 and FP16, K = 192 .. 1536,
+  // n_out = 192 .. 3072, T = 6272 .. 100352): the pair is the faster kernel whenever its
+  // 256-channel tiles are whole (an even number of 128-channel tiles; with an odd number the
+  // last pair computes a padding tile, a quarter or more of the work at the ViT and Swin
+  // widths) and there are at least as many 256 x 128 pair tiles as SMs (fewer, and the single-SM
+  // kernel's smaller tiles balance better); by 5-25 % at K = 768 .. 1536, as its operand bytes
+  // in flight per SM pair and its single MMA issuer outweigh the streaming kernel's shorter
+  // tiles.  A long k loop (>= 2 KB of X per token) takes it regardless: per-stage issue cost
+  // and X re-reads dominate there.
+  const int64_t kbytes = h->k * nm::elem_bytes(h->dt);
+  const bool pair_default = kbytes >= 2048 ||
+                            (kbytes >= 192 && h->n_ct % 2 == 0 && (int64_t)(h->n_ct / 2) * ((T + 127) / 128) >= sms);
   if ((forced_pair == 1 || (forced_pair == -1 && pair_default)) && forced_split <= 1 && forced_xs != 1) {
     const int cands[3] = {224, 192, 128};
     double best_cost = 1e300;

@@ -857,6 +857,9 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
 #pragma unroll 1
         for (int c = 0; c < C::NCH; ++c) {
           uint32_t r[C::CH];
+          // tcgen05.ld is .sync.aligned: reconverge after the previous chunk's
+          // per-lane stores (and lane 0's tensor store) before issuing it
+          __syncwarp();
           tmem_ld_n<C::CH>(tbase + (uint32_t)(c * C::CH), r);
           tmem_wait_ld();
           if (c == C::NCH - 1) {  // all of this warp's columns are in registers: release the accumulator
@@ -1013,7 +1016,11 @@ __global__ void __launch_bounds__(kernel_threads(IMG, OUT), 1)
 // issues every MMA for both SMs, which halves the per-SM cost of MMA issue, and
 // each SM loads only half of the X tile.  Both CTAs' copies count on the
 // leader's stage barrier; the leader's commits arrive on both CTAs' barriers;
-// the peer's epilogue releases accumulators with remote arrives on the leader.
+// the peer's epilogue releases accumulators through its own warp 1, which
+// forwards one cluster-scope arrive per release to the leader.  (A cluster-scope
+// release issued by an epilogue lane would first wait for that lane's own
+// output stores to become visible, holding the leader's next tile back by the
+// store latency; the forwarding warp has no stores in flight.)
 // No load uses cluster multicast.
 template <int DT, int IMG, int BN, int OUT>
 struct PairCfg {
@@ -1064,6 +1071,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
   __shared__ __align__(8) uint64_t accf_bar[2];
   __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ __align__(8) uint64_t pfree_bar[2];  // peer: its epilogue warps have read accumulator i
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
@@ -1081,7 +1089,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accf_bar[i], 1);
-      mbar_init(&acce_bar[i], 2 * C::EPI_WARPS);  // both CTAs' epilogue warps release the leader's accumulator
+      // the leader's epilogue warps, plus one arrive forwarded by the peer for
+      // all of its warps (tensor-store variant: every peer warp arrives itself)
+      mbar_init(&acce_bar[i], C::TS ? 2 * C::EPI_WARPS : C::EPI_WARPS + 1);
+      mbar_init(&pfree_bar[i], C::EPI_WARPS);
     }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -1239,7 +1250,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
       if (issuer) tc_commit_pair(&drain_bar, (uint16_t)3);  // every MMA of this pair has completed
       mbar_wait_warp(&drain_bar, 0, &abort_sh, tmo);
     } else {
-      mbar_wait_warp(&drain_bar, 0, &abort_sh, tmo);  // peer: the leader's MMAs into this TMEM are done
+      // Peer: forward each accumulator release of this CTA's epilogue to the
+      // leader.  The epilogue warps arrive on a local barrier (no wait for
+      // their own output stores to drain); this warp, with no stores of its own
+      // in flight, turns each completed phase into one cluster-scope release on
+      // the leader's barrier (releases are cumulative, so the epilogue's tensor
+      // memory reads, fenced before its local arrives, are ordered before it).
+      // The tensor-store variant's epilogue arrives on the leader itself: its
+      // output leaves through asynchronous bulk copies, which a release does not
+      // wait for.
+      if constexpr (!C::TS) {
+        const bool issuer = elect_one();
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = u_first; u < a.units; u += u_step) {
+          if (!mbar_wait_warp(&pfree_bar[acc], acc_phase, &abort_sh, tmo)) {
+            if (issuer) give_up(4);
+            break;
+          }
+          if (issuer) mbar_arrive_cluster(acce_lead0 + 8u * (uint32_t)acc);
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
+      }
+      mbar_wait_warp(&drain_bar, 0, &abort_sh, tmo);  // the leader's MMAs into this TMEM are done
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
@@ -1273,16 +1309,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(cta_threads(OUT), 1)
 #pragma unroll 1
       for (int c = 0; c < C::NCH; ++c) {
         uint32_t r[C::CH];
+        __syncwarp();  // tcgen05.ld is .sync.aligned: reconverge after the previous chunk's stores
         tmem_ld_n<C::CH>(tbase + (uint32_t)(c * C::CH), r);
         tmem_wait_ld();
-        if (c == C::NCH - 1) {  // release the accumulator on the leader
+        if (c == C::NCH - 1) {  // release the accumulator (the peer's release is forwarded by its warp 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
             if (leader)
               mbar_arrive(&acce_bar[acc]);
-            else
+            else if constexpr (C::TS)
               mbar_arrive_cluster(acce_lead0 + 8u * (uint32_t)acc);
+            else
+              mbar_arrive(&pfree_bar[acc]);
           }
         }
         const int tc0 = t0 + c * C::CH;
