@@ -1084,7 +1084,7 @@ def main() -> None:
 def _kernel_sha() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("nm_spmm.cu", "nm_device.cuh"):
+    for f in ("nm_spmm.cu", "nm_device.cuh", "nm_api.cu"):  # the kernels and the planner that picks them
         h.update(open(os.path.join(ROOT, "structured_sparse_gemm_compress_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

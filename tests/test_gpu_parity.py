@@ -288,6 +288,45 @@ def test_planner_splits_small_token_counts_on_chip(n_out, K, N, M):
         assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32)), T
 
 
+@pytest.mark.parametrize("dtype,K,n_out,T,want", [
+    ("int8", 768, 768, 12608, 1),     # 6 channel tiles, 3 x 99 pair tiles
+    ("int8", 768, 2304, 12608, 1),
+    ("int8", 768, 384, 12608, 0),     # 3 channel tiles: the last pair would compute a padding tile
+    ("int8", 768, 576, 100352, 0),    # 5 channel tiles
+    ("int8", 768, 192, 12608, 0),     # 1 x 99 pair tiles, fewer than the SMs
+    ("int8", 768, 768, 6272, None),   # 3 x 49 = 147 pair tiles: pair iff the GPU has <= 147 SMs
+    ("int8", 96, 768, 100352, 0),     # under 192 bytes of X per token
+    ("int8", 3072, 384, 12608, 1),    # >= 2 KB of X per token: pair whatever the tile count
+    ("fp16", 768, 768, 6304, 1),      # 1536 bytes per token, 3 x 50 pair tiles
+])
+def test_planner_pair_rule(dtype, K, n_out, T, want):
+    """The planner takes the two-SM kernel when its 256-channel tiles are whole
+    (an even count of 128-channel tiles) and there are at least as many 256 x
+    128 pair tiles as SMs (K*b >= 192 bytes), or when a token row of X is at
+    least 2 KB."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if want is None:
+        want = int(3 * 49 >= sms)
+    h = nm.nm_compress(_weights(dtype, n_out, K, seed=441).cuda(), 2, 4)
+    assert nm.nm_plan_query(h, T, scaled=True)["pair"] == want
+
+
+@pytest.mark.parametrize("n_out,want_pair", [(256, 1), (384, 0), (250, 1)])
+def test_planner_pair_rule_parity(monkeypatch, n_out, want_pair):
+    """The same rule on a GPU capped at 16 persistent CTAs (16 pair tiles are
+    enough), and the output of whichever kernel it picks is the oracle's."""
+    monkeypatch.setenv("NMSPMM_FORCE_GRID", "16")
+    T, K = 2000, 768
+    W = _weights("int8", n_out, K, seed=451)
+    X = _acts("int8", T, K, seed=452)
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=453)
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    assert nm.nm_plan_query(h, T, scaled=True)["pair"] == want_pair
+    Y = nm.nm_spmm(h, X.cuda(), scale=s.cuda())
+    ref = oracle.spmm(X.numpy(), W.numpy(), 2, 4, scale=s.numpy())
+    assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
 @pytest.mark.parametrize("grid", ["5", "148"])
 @pytest.mark.parametrize("N,M", [(2, 4), (1, 4), (2, 8), (4, 8), (4, 4)])
 @pytest.mark.parametrize("T,n_out,K", [(1000, 300, 768), (129, 200, 512), (640, 384, 256)])
