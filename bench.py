@@ -853,24 +853,30 @@ def main() -> None:
 
     pack_stream = torch.cuda.Stream()
     packed = [torch.cuda.Event() for _ in ls]  # re-pack of problem i done
+    used = [torch.cuda.Event() for _ in ls]    # SpMM of problem i done (its packed image is free)
 
-    def step(st=None, ps=None):
+    def step(st=None, ps=None, first=True):
         """One pass over the 16 problems: per (layer, N:M) a re-pack of the weight
-        on a second stream and the SpMM on the main stream.  The re-packs follow
-        everything issued before the step on the main stream (input copies, the
-        previous step's SpMMs on the same handles); each SpMM waits only for its
-        own re-pack, so the re-packs of later problems run under earlier SpMMs."""
+        on a second stream and the SpMM on the main stream.  The first step of a
+        sequence re-packs after everything issued before it on the main stream
+        (input copies, earlier work); a later step's re-pack of problem i waits
+        only for the previous step's SpMM i, the one reader of that packed image.
+        Each SpMM waits only for its own re-pack, so re-packs run under the
+        SpMMs of other problems, across step boundaries too."""
         st = stream if st is None else st
         ps = pack_stream if ps is None else ps
-        ps.wait_stream(st)
+        if first:
+            ps.wait_stream(st)
         for i, l in enumerate(ls):
+            if not first:
+                ps.wait_event(used[i])
             nm.nm_recompress(handles[i], devb[l.name]["W"], stream=ps)
             packed[i].record(ps)
         for i, l in enumerate(ls):
             d = devb[l.name]
             st.wait_event(packed[i])
             nm.nm_spmm(handles[i], d["X"], Y=Ys[i], scale=d["s"], stream=st)
-        st.wait_stream(ps)
+            used[i].record(st)
 
     for _ in range(args.warmup):
         step()
@@ -895,7 +901,7 @@ def main() -> None:
             cap.wait_stream(stream)
             with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
                 for k in range(n):
-                    step(st=cap, ps=cap_pack)
+                    step(st=cap, ps=cap_pack, first=k == 0)
             g.replay()  # upload + one untimed pass
             built[n] = g
         graphs = [built[n] for n in sizes]
@@ -913,7 +919,7 @@ def main() -> None:
                 clk.poke()
         else:
             for k in range(args.steps):
-                step()
+                step(first=k == 0)
         stop.record(stream)
         clk.poke()
         torch.cuda.synchronize()

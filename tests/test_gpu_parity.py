@@ -372,6 +372,37 @@ def test_cta_pair_bit_exact(monkeypatch, bn, grid, N, M, T, n_out, K, tma_store)
         assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
 
 
+@pytest.mark.parametrize("tma_store", ["0", "1"])
+def test_cta_pair_repeated_calls_few_clusters(monkeypatch, tma_store):
+    """Accumulator hand-over between the two CTAs of a pair under load: six
+    clusters walk 12 tiles each, so every accumulator is released and refilled
+    six times per call; 30 calls, alternating the fp32 and int32 outputs, must
+    all be bit-exact and end without a timed-out wait."""
+    monkeypatch.setenv("NMSPMM_TMA_STORE", tma_store)
+    monkeypatch.setenv("NMSPMM_FORCE_PAIR", "1")
+    monkeypatch.setenv("NMSPMM_FORCE_BN", "128")
+    monkeypatch.setenv("NMSPMM_FORCE_GRID", "12")
+    T, n_out, K = 4500, 512, 768  # 2 channel-tile pairs x 36 token tiles = 72 pair tiles
+    W = _weights("int8", n_out, K, seed=461)
+    X = _acts("int8", T, K, seed=462)
+    s = inputs.scale_uniform(n_out, 0.001, 0.01, seed=463)
+    refs = {True: oracle.spmm(X.numpy(), W.numpy(), 2, 4, scale=s.numpy()),
+            False: oracle.spmm(X.numpy(), W.numpy(), 2, 4)}
+    h = nm.nm_compress(W.cuda(), 2, 4)
+    plan = nm.nm_plan_query(h, T, scaled=True)
+    assert plan["pair"] == 1 and plan["grid"] == 6
+    Xd, sd = X.cuda(), s.cuda()
+    bad = []
+    for i in range(30):
+        scaled = i % 2 == 0
+        Y = nm.nm_spmm(h, Xd, scale=sd if scaled else None)
+        torch.cuda.synchronize()
+        assert nm.nm_device_status(h) == nm.NM_OK, i
+        if not np.array_equal(Y.cpu().numpy().view(np.uint32), refs[scaled].view(np.uint32)):
+            bad.append(i)
+    assert not bad, bad
+
+
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("bn", ["128", "224"])
 @pytest.mark.parametrize("N,M", [(2, 4), (2, 8), (4, 8)])
