@@ -40,7 +40,7 @@ from structured_sparse_gemm_compress_b200 import inputs  # noqa: E402
 METRIC = "N:M SpMM effective TOPS (dense-equiv) on ViT-B layers; % of sparse-TC roofline"
 UNIT = "TOPS"
 WORKLOAD = "ViT-B/16 INT8 linear set, batch 64 (T=12608), N:M in {1:4,2:4,2:8,4:8}, per-channel fp32 scale"
-CPU_SAMPLE_ROWS = 1536      # about 10-30 s of oracle work on the host cores
+CPU_SAMPLE_ROWS = 9216      # ~10 s of oracle work on a 16-thread host (1536 rows took 1.7 s there)
 REF_SAMPLE_ROWS = 192       # per reference-arm step, so --steps 20 stays within a few minutes
 
 
