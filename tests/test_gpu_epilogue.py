@@ -6,8 +6,9 @@ fp32 / fp16 / bf16 (round to nearest even) or int8 (round half to even of
 y * out_scale, saturated).
 
 * INT8 handle, no activation: every output type is bit-exact.
-* GELU: the kernel evaluates erf with the device's fp32 erff (at most 2 ulp),
-  the oracle in fp64, so results agree within
+* GELU: the kernel evaluates erf by Abramowitz and Stegun's formula 7.1.26
+  (absolute error at most 1.5e-7) with the hardware's approximate reciprocal
+  and power of two, the oracle in fp64, so results agree within
       |y - g| <= 4e-7 |v| + 2e-6 |g|   (v the value before GELU, g = GELU(v))
   plus the output type's own rounding; an int8 code may differ by one only
   where the oracle's unrounded value lies that close to a half-integer.
