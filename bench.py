@@ -160,11 +160,14 @@ class ClockSampler:
 
 
 class NvmlSampler:
-    """SM clock, its maximum, power and clock-event reasons of the GPU this
+    """SM clock, its maximum and the clock-event reasons of the GPU this
     process uses (found by PCI bus id), polled by NVML from a thread about
-    every millisecond between ``mark_start`` and ``mark_end``, so even a timed
-    region of a few milliseconds is covered.  Falls back to ``ClockSampler``
-    (nvidia-smi every 50 ms) when NVML is unavailable."""
+    every half millisecond between ``mark_start`` and ``mark_end``, so even a
+    timed region of a few milliseconds is covered.  The power draw is read only
+    just before and just after the region: on B200 an NVML power reading taken
+    while the GPU was busy stretched a 20-step region up to 7x (clock and reason
+    readings did not).  Falls back to ``ClockSampler`` (nvidia-smi every 50 ms)
+    when NVML is unavailable."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
@@ -172,6 +175,7 @@ class NvmlSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.samples = []
+        self.power = []
         self._run = False
         self._thread = None
         self._nvml = None
@@ -209,8 +213,13 @@ class NvmlSampler:
         try:
             sm = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
             rs = get_reasons(self._h)
-            pw = n.nvmlDeviceGetPowerUsage(self._h) / 1000.0 if len(self.samples) % 8 == 0 else None
-            self.samples.append((sm, rs, pw))
+            self.samples.append((sm, rs, None))
+        except Exception:
+            pass
+
+    def _power(self):
+        try:
+            self.power.append(self._nvml.nvmlDeviceGetPowerUsage(self._h) / 1000.0)
         except Exception:
             pass
 
@@ -218,6 +227,7 @@ class NvmlSampler:
         while self._run:
             if self._inside:
                 self._sample()
+                time.sleep(0.0005)
             else:
                 time.sleep(0.0002)
 
@@ -229,12 +239,14 @@ class NvmlSampler:
     def mark_start(self):
         if self._fallback is not None:
             return self._fallback.mark_start()
+        self._power()
         self._inside = True
 
     def mark_end(self):
         if self._fallback is not None:
             return self._fallback.mark_end()
         self._inside = False
+        self._power()
 
 
 
@@ -253,10 +265,11 @@ class NvmlSampler:
                     "samples": 0, "samples_in_timed_region": 0, "source": "nvml"}
         sm = [x[0] for x in self.samples]
         reasons = sorted({name for _, rs, _ in self.samples for name, bit in self.REASONS if rs & bit})
-        pw = [x[2] for x in self.samples if x[2] is not None]
         return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "power_w_max": round(max(pw), 1) if pw else None,
-                "samples": len(sm), "samples_in_timed_region": len(sm), "source": "nvml, ~1 ms polling"}
+                "reasons": reasons, "power_w_max": round(max(self.power), 1) if self.power else None,
+                "power_read": "just before and just after the timed region",
+                "samples": len(sm), "samples_in_timed_region": len(sm),
+                "source": "nvml clocks and reasons, ~0.5 ms polling"}
 
 
 # --------------------------------------------------------------------------- multi-rank plumbing
