@@ -164,8 +164,11 @@ nm_status nm_spmm(const nm_handle* h, const void* X_dev, int64_t T, void* Y_dev,
  *   NM_OUT_DEFAULT                  INT8: INT32 when scale, bias and act are
  *                                   all absent, else FP32; FP16/BF16: the
  *                                   input's type.
- * With act == NM_ACT_NONE and an INT8 handle the result is exactly fixed; the
- * GELU uses the device's erff, so it is within erff's error bound.
+ * With act == NM_ACT_NONE and an INT8 handle the result is exactly fixed.  The
+ * GELU evaluates erf by formula 7.1.26 of Abramowitz and Stegun (absolute error
+ * at most 1.5e-7) with the GPU's approximate reciprocal and power of two; the
+ * GELU value g of a pre-activation v is within 4e-7 |v| + 2e-6 |GELU(v)| of the
+ * exact one.
  */
 typedef enum {
   NM_OUT_DEFAULT = 0,
