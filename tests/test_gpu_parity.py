@@ -372,13 +372,15 @@ def test_cta_pair_bit_exact(monkeypatch, bn, grid, N, M, T, n_out, K, tma_store)
         assert np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("tma_store", ["0", "1"])
+@pytest.mark.parametrize("tma_store", ["0", "1", "runtime-stage"])
 def test_cta_pair_repeated_calls_few_clusters(monkeypatch, tma_store):
     """Accumulator hand-over between the two CTAs of a pair under load: six
     clusters walk 12 tiles each, so every accumulator is released and refilled
-    six times per call; 30 calls, alternating the fp32 and int32 outputs, must
-    all be bit-exact and end without a timed-out wait."""
-    monkeypatch.setenv("NMSPMM_TMA_STORE", tma_store)
+    six times per call; 30 calls, alternating scaled and unscaled outputs (the
+    fixed stages: fp32 and int32; the runtime stage: fp32 with a zero bias),
+    must all be bit-exact and end without a timed-out wait."""
+    runtime = tma_store == "runtime-stage"  # the output stage read from the launch (nm_spmm_ex)
+    monkeypatch.setenv("NMSPMM_TMA_STORE", "0" if runtime else tma_store)
     monkeypatch.setenv("NMSPMM_FORCE_PAIR", "1")
     monkeypatch.setenv("NMSPMM_FORCE_BN", "128")
     monkeypatch.setenv("NMSPMM_FORCE_GRID", "12")
@@ -392,9 +394,18 @@ def test_cta_pair_repeated_calls_few_clusters(monkeypatch, tma_store):
     plan = nm.nm_plan_query(h, T, scaled=True)
     assert plan["pair"] == 1 and plan["grid"] == 6
     Xd, sd = X.cuda(), s.cuda()
+    zero = torch.zeros(n_out, dtype=torch.float32, device="cuda")
     bad = []
     for i in range(30):
         scaled = i % 2 == 0
+        if runtime:  # a (zero) bias routes the call to the runtime stage; fp32 out with and without the scale
+            Y = nm.nm_spmm_ex(h, Xd, scale=sd if scaled else None, bias=zero, out="float32")
+            ref = refs[scaled] if scaled else refs[False].astype(np.float32)
+            torch.cuda.synchronize()
+            assert nm.nm_device_status(h) == nm.NM_OK, i
+            if not np.array_equal(Y.cpu().numpy().view(np.uint32), ref.view(np.uint32)):
+                bad.append(i)
+            continue
         Y = nm.nm_spmm(h, Xd, scale=sd if scaled else None)
         torch.cuda.synchronize()
         assert nm.nm_device_status(h) == nm.NM_OK, i
