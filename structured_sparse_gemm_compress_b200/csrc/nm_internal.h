@@ -121,8 +121,8 @@ struct SpmmArgs {
 // slots: [kind][index], kinds below, kTraceMax indices each.
 constexpr int kTraceMax = 64;
 // TR_GT holds %globaltimer (ns, comparable across SMs) at kernel entry (0),
-// after the wait on the previous kernel (1), after the role loops (2) and at
-// exit (3), written by thread 0.
+// after the wait on the previous kernel (1), after the producer's loop (2) and
+// at exit (3), written by thread 0, and the SM clock at the same points (4..7).
 enum : int { TR_P_ISSUE = 0, TR_M_FULL, TR_M_DONE, TR_M_ACCE, TR_E_START, TR_E_END, TR_GT, TR_KINDS };
 constexpr int kTraceStride = TR_KINDS * kTraceMax;
 

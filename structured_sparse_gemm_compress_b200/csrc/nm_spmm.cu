@@ -150,8 +150,11 @@ __host__ __device__ constexpr uint32_t make_idesc() {
   } while (0)
 #define NM_TG(idx)                                                                                   \
   do {                                                                                               \
-    if (a.trace && threadIdx.x == 0)                                                                 \
-      a.trace[(size_t)blockIdx.x * kTraceStride + TR_GT * kTraceMax + (idx)] = (long long)globaltimer(); \
+    if (a.trace && threadIdx.x == 0) {                                                               \
+      long long* g_ = a.trace + (size_t)blockIdx.x * kTraceStride + TR_GT * kTraceMax;               \
+      g_[(idx)] = (long long)globaltimer();                                                          \
+      g_[4 + (idx)] = (long long)clock64();                                                          \
+    }                                                                                                \
   } while (0)
 #else
 #define NM_TR(kind, idx) \

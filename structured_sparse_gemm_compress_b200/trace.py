@@ -108,6 +108,10 @@ def run(problems: list[str], raw_out: bool = False) -> dict:
         raw = {f"cta{b}": {k: [int(x) for x in tr[b, i, :24]] for i, k in
                            enumerate(("p_issue", "m_full", "m_done", "m_acce", "e_start", "e_end"))}
                for b in (0, 1) if b < tr.shape[0]}
+        for b in (0, 1):
+            if b < tr.shape[0]:
+                raw[f"cta{b}"]["gt_ns"] = [int(x - base) for x in tr[b, GT, :4]]
+                raw[f"cta{b}"]["gt_clk"] = [int(x) for x in tr[b, GT, 4:8]]
         r = {"problem": p["name"], "plan": p["plan"], **_stage_stats(tr, bool(p["plan"]["pair"])),
              "entry_us": round((gt[:, 0].min() - base) / 1e3, 2), "first_wait_return_us": round((gt[:, 1].min() - base) / 1e3, 2),
              "exit_first_us": round((gt[:, 3].min() - base) / 1e3, 2), "exit_last_us": round((gt[:, 3].max() - base) / 1e3, 2)}
