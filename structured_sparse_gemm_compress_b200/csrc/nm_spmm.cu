@@ -1167,11 +1167,19 @@ struct PairCfg {
   static constexpr int EPI_WARPS = epi_warps(OUT);
   static constexpr int THREADS = cta_threads(OUT);
   static constexpr int WCOLS = BN / (EPI_WARPS / 4);  // token columns per epilogue warp
-  static constexpr int CH = (WCOLS % 32 == 0) ? 32 : (WCOLS % 16 == 0) ? 16 : 8;
+  static constexpr bool TS = (OUT & kOutDirect) == 0;
+  // Columns per tcgen05.ld run: 32, or, for the INT8 fixed output stages with
+  // direct stores, half of a warp's columns when they are not a multiple of 32
+  // (224-token tiles: two runs of 56 rather than seven of 16; measured 4-5 %
+  // faster on the ViT-B qkv layers, and 1.5 % slower for the FP16 kernels,
+  // which keep the short runs).
+  static constexpr int CH = (WCOLS % 32 == 0) ? 32
+                            : (DT == DT_I8 && !TS && (OUT & kOutEpi) == 0 && WCOLS <= 112 && (WCOLS / 2) % 8 == 0)
+                                ? WCOLS / 2
+                                : (WCOLS % 16 == 0) ? 16 : 8;
   static constexpr int NCH = WCOLS / CH;
   static constexpr int OES = out_bytes(OUT);
   static constexpr int EPI_BUF = CH * 32 * OES;
-  static constexpr bool TS = (OUT & kOutDirect) == 0;
   static constexpr int EPI_NB = (kSmemBudget - 2 * EPI_WARPS * EPI_BUF) / STAGE >= 4 ? 2 : 1;
   static constexpr int EPI_BYTES = TS ? EPI_NB * EPI_WARPS * EPI_BUF : 0;
   static constexpr int STAGES_FIT = (kSmemBudget - EPI_BYTES) / STAGE;
