@@ -303,6 +303,27 @@ typedef struct nm_plan_info {
 } nm_plan_info;
 nm_status nm_plan_query(const nm_handle* h, int64_t T, int scaled, nm_plan_info* out);
 
+/*
+ * nm_plan_for_shape -- test and diagnostic hook (no counterpart in the paper):
+ * the plan nm_plan_query would report for a handle of this shape (nm_compress
+ * with dt, n_out, k, N, M) and T tokens on a GPU with `sms` SMs whose
+ * resident-cluster capacities are given instead of queried, so the planner's
+ * rules can be checked without a GPU.  Touches no device and allocates
+ * nothing.
+ *
+ * pair_clusters    int[3]: CTA pairs of the two-SM kernel that fit on the GPU
+ *                  at the token tiles 224, 192 and 128 (<= 0: that tile cannot
+ *                  run); nm_plan_query queries these from the device for the
+ *                  output the call would write.
+ * stream_clusters  int[8]: clusters of S one-SM CTAs that fit, S = 1 .. 8
+ *                  (<= 0: none).
+ * The NMSPMM_FORCE_* environment overrides apply as in nm_spmm.  Errors:
+ * NM_ERR_INVALID for null pointers, a bad dtype, shape, T or sms;
+ * NM_ERR_UNSUPPORTED for an N:M nm_compress rejects.
+ */
+nm_status nm_plan_for_shape(nm_dtype dt, int64_t n_out, int64_t k, int N, int M, int64_t T, int sms,
+                            const int* pair_clusters, const int* stream_clusters, nm_plan_info* out);
+
 /* nm_query -- shape and format of a handle; any output pointer may be NULL. */
 nm_status nm_query(const nm_handle* h, int64_t* n_out, int64_t* k, int* N, int* M, nm_dtype* dt);
 

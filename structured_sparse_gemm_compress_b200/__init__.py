@@ -26,7 +26,8 @@ _ELEM = {NM_INT8: torch.int8, NM_FP16: torch.float16, NM_BF16: torch.bfloat16}
 # Every symbol include/nmspmm.h declares.
 EXPORTS = ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_ex", "nm_spmm_gather",
            "nm_spmm_gather_ex", "nm_spmm_noalloc", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
-           "nm_plan_query", "nm_device_status", "nm_destroy", "nm_last_error", "nm_version", "nm_test_spmm_skip_stage")
+           "nm_plan_query", "nm_plan_for_shape", "nm_device_status", "nm_destroy", "nm_last_error", "nm_version",
+           "nm_test_spmm_skip_stage")
 
 
 class NMPlanInfo(ctypes.Structure):
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.nm_query.argtypes = [vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i32),
                                ctypes.POINTER(i32), ctypes.POINTER(i32)]
         L.nm_plan_query.argtypes = [vp, i64, i32, ctypes.POINTER(NMPlanInfo)]
+        L.nm_plan_for_shape.argtypes = [i32, i64, i64, i32, i32, i64, i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                        ctypes.POINTER(NMPlanInfo)]
         L.nm_device_status.argtypes = [vp]
         L.nm_destroy.argtypes = [vp]
         L.nm_destroy.restype = None
@@ -76,7 +79,7 @@ def lib() -> ctypes.CDLL:
         for name in ("nm_compress", "nm_compress_tile", "nm_recompress", "nm_spmm", "nm_spmm_gather",
                      "nm_spmm_gather_ex", "nm_spmm_noalloc",
                      "nm_test_spmm_skip_stage", "nm_decompress", "nm_export", "nm_export_sizes", "nm_query",
-                     "nm_plan_query", "nm_device_status"):
+                     "nm_plan_query", "nm_plan_for_shape", "nm_device_status"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -326,6 +329,22 @@ def nm_plan_query(h: NMHandle, T: int, scaled: bool = False) -> dict:
     """The launch plan the SpMM call would use for T tokens (kernel, token tile, splits, cluster, grid)."""
     info = NMPlanInfo()
     _check(lib().nm_plan_query(h.raw, int(T), int(bool(scaled)), ctypes.byref(info)))
+    return {f: getattr(info, f) for f, _ in NMPlanInfo._fields_}
+
+
+def nm_plan_for_shape(dtype: torch.dtype, n_out: int, k: int, N: int, M: int, T: int, sms: int,
+                      pair_clusters=(74, 74, 74), stream_clusters=(148, 74, 48, 37, 28, 24, 21, 18)) -> dict:
+    """The plan nm_plan_query would report for a handle of this shape on a GPU
+    with ``sms`` SMs and the given resident-cluster capacities (two-SM kernel
+    pairs at token tiles 224/192/128; clusters of 1..8 one-SM CTAs).  Needs no
+    GPU: a test and diagnostic hook of the planner."""
+    if dtype not in _TORCH_DT or len(pair_clusters) != 3 or len(stream_clusters) != 8:
+        raise ValueError("dtype must be int8/float16/bfloat16, pair_clusters 3 values, stream_clusters 8")
+    pc = (ctypes.c_int * 3)(*[int(v) for v in pair_clusters])
+    sc = (ctypes.c_int * 8)(*[int(v) for v in stream_clusters])
+    info = NMPlanInfo()
+    _check(lib().nm_plan_for_shape(_TORCH_DT[dtype], int(n_out), int(k), int(N), int(M), int(T), int(sms), pc, sc,
+                                   ctypes.byref(info)))
     return {f: getattr(info, f) for f, _ in NMPlanInfo._fields_}
 
 

@@ -201,6 +201,26 @@ int out_code(const nm_handle* h, bool scaled) {
   return h->dt == nm::DT_F16 ? nm::OUT_F16 : nm::OUT_BF16;
 }
 
+// Resident-cluster capacities the planner consults: queried from the device
+// (device_capacity), or given by the caller of nm_plan_for_shape so that the
+// planner's rules can be exercised without a GPU.
+struct Capacity {
+  int pair[3] = {0, 0, 0};                // resident CTA pairs of the two-SM kernel, token tiles 224 / 192 / 128
+  int stream[nm::kMaxClusterSplit + 1] = {};  // [S]: resident clusters of S one-SM CTAs (S = 1 .. 8)
+};
+
+constexpr int kPairTiles[3] = {224, 192, 128};
+
+int pair_slot(int bn) { return bn == 224 ? 0 : bn == 192 ? 1 : 2; }
+
+Capacity device_capacity(const nm_handle* h, bool scaled) {
+  Capacity c;
+  if (!h->tile)
+    for (int i = 0; i < 3; ++i) c.pair[i] = nm::pair_max_clusters(h->dt, h->img, kPairTiles[i], out_code(h, scaled));
+  for (int S = 1; S <= nm::kMaxClusterSplit; ++S) c.stream[S] = nm::stream_max_clusters(S);
+  return c;
+}
+
 // Small-token model of one streaming launch (us), fitted on B200 to a sweep of
 // forced (token tile, split) plans over the ViT-B INT8 shapes at T = 16 .. 788
 // (CUDA graphs of back-to-back launches; within ~5 % of every point):
@@ -219,13 +239,13 @@ struct SmallTModel {
   double l2_bytes_per_us = 10.0e6;  // aggregate L2 -> SM operand rate (~10 TB/s)
 };
 
-double small_t_cost(const nm_handle* h, int64_t T, int sms, int bn, int S) {
+double small_t_cost(const nm_handle* h, int64_t T, int sms, int bn, int S, const Capacity& capacity) {
   const SmallTModel m;
   const int64_t tiles = (int64_t)h->n_ct * ((T + bn - 1) / bn);
   const int kbs = (h->n_kb + S - 1) / S;
   int64_t cap = sms;  // tiles resident at once: one per SM, or one per resident cluster
   if (S > 1) {
-    const int c = nm::stream_max_clusters(S);
+    const int c = capacity.stream[S];
     if (c <= 0) return 1e300;
     cap = c;
   }
@@ -243,14 +263,15 @@ double small_t_cost(const nm_handle* h, int64_t T, int sms, int bn, int S) {
 // is clearly faster; then sets both.  (Measured: at T <= 64 the K = 3072 ViT-B
 // layer drops from 5.8 to 4.8 us with 6 splits of 32-token tiles; K = 768
 // layers, whose 3 k-blocks leave nothing to split, stay unsplit.)
-void choose_cluster_split(const nm_handle* h, int64_t T, int sms, int forced_bn, nm::Plan* p, int* splits) {
-  double best = small_t_cost(h, T, sms, p->bn, 1);
+void choose_cluster_split(const nm_handle* h, int64_t T, int sms, int forced_bn, const Capacity& capacity, nm::Plan* p,
+                          int* splits) {
+  double best = small_t_cost(h, T, sms, p->bn, 1, capacity);
   for (int bn : {32, 64, 128}) {
     if (forced_bn && bn != forced_bn) continue;
     for (int S = 2; S <= std::min(nm::kMaxClusterSplit, h->n_kb); ++S) {
       const int kps = (h->n_kb + S - 1) / S;
       if ((h->n_kb + kps - 1) / kps != S) continue;  // every split owns >= 1 k-block
-      const double c = small_t_cost(h, T, sms, bn, S);
+      const double c = small_t_cost(h, T, sms, bn, S, capacity);
       if (c < best * 0.95) {  // a clear win only
         best = c;
         p->bn = bn;
@@ -261,8 +282,9 @@ void choose_cluster_split(const nm_handle* h, int64_t T, int sms, int forced_bn,
 }
 
 // Adaptive parallelism: pick the kernel (CTA pair or single SM), the token tile
-// and the split-K factor for this shape (rules and their measurements below).
-nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
+// and the split-K factor for this shape (rules and their measurements below),
+// given the resident-cluster capacities.
+nm::Plan plan_with(const nm_handle* h, int64_t T, int sms, const Capacity& capacity) {
   nm::Plan p;
   const int forced_bn = env_int("NMSPMM_FORCE_BN", 0);
   const int forced_split = env_int("NMSPMM_FORCE_SPLITK", 0);
@@ -310,7 +332,7 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
     double best_cost = 1e300;
     for (int bn : cands) {
       if (forced_bn && bn != forced_bn) continue;
-      int clusters = nm::pair_max_clusters(h->dt, h->img, bn, out_code(h, scaled));
+      int clusters = capacity.pair[pair_slot(bn)];
       if (clusters <= 0) continue;
       if (forced_grid > 0) clusters = std::min(clusters, std::max(1, forced_grid / 2));
       const int64_t units = (int64_t)((h->n_ct + 1) / 2) * ((T + bn - 1) / bn);
@@ -374,7 +396,7 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
     // CTAs of a cluster, which sum their partials on chip (no workspace), when
     // the model below says that beats the unsplit tile.
     const int64_t tiles0 = (int64_t)h->n_ct * ((T + p.bn - 1) / p.bn);
-    if (tiles0 < sms) choose_cluster_split(h, T, sms, forced_bn, &p, &splits);
+    if (tiles0 < sms) choose_cluster_split(h, T, sms, forced_bn, capacity, &p, &splits);
   }
   p.n_tt = (int)((T + p.bn - 1) / p.bn);
   const int64_t tiles = (int64_t)h->n_ct * p.n_tt;
@@ -388,11 +410,16 @@ nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
   // workspace reduction is asked for (NMSPMM_SPLIT_GLOBAL=1) or the split is
   // wider than a portable cluster.
   if (p.splits > 1 && p.splits <= nm::kMaxClusterSplit && env_int("NMSPMM_SPLIT_GLOBAL", 0) == 0 &&
-      nm::stream_max_clusters(p.splits) > 0) {
+      capacity.stream[p.splits] > 0) {
     p.cluster = 1;
     p.grid = p.units;
   }
   return p;
+}
+
+// The plan for a call on this handle's device.
+nm::Plan make_plan(const nm_handle* h, int64_t T, int sms, bool scaled) {
+  return plan_with(h, T, sms, device_capacity(h, scaled));
 }
 
 nm_status check_handle(const nm_handle* h) {
@@ -910,6 +937,40 @@ nm_status nm_plan_query(const nm_handle* h, int64_t T, int scaled, nm_plan_info*
   if (!out) return fail(NM_ERR_INVALID, "null output");
   if (T <= 0 || T > INT32_MAX) return fail(NM_ERR_INVALID, "T must be in [1, 2^31-1] (got %lld)", (long long)T);
   const nm::Plan p = make_plan(h, T, num_sms(h->device), scaled != 0);
+  out->pair = p.pair;
+  out->bn = p.bn;
+  out->splits = p.splits;
+  out->cluster = p.cluster;
+  out->grid = p.grid;
+  out->units = p.units;
+  return NM_OK;
+}
+
+nm_status nm_plan_for_shape(nm_dtype dt, int64_t n_out, int64_t k, int N, int M, int64_t T, int sms,
+                            const int* pair_clusters, const int* stream_clusters, nm_plan_info* out) {
+  g_err.clear();
+  if (!pair_clusters || !stream_clusters || !out) return fail(NM_ERR_INVALID, "null argument");
+  if (dt != NM_INT8 && dt != NM_FP16 && dt != NM_BF16) return fail(NM_ERR_INVALID, "unknown dtype %d", (int)dt);
+  if (n_out <= 0 || k <= 0 || n_out > INT32_MAX || k > INT32_MAX) return fail(NM_ERR_INVALID, "bad shape");
+  const bool sp24 = (N == 1 && M == 4) || (N == 2 && M == 4) || (N == 2 && M == 8);
+  const bool dense = (N == 4 && M == 8) || (N == M && (M == 4 || M == 8));
+  if (!sp24 && !dense) return fail(NM_ERR_UNSUPPORTED, "N:M %d:%d is not supported", N, M);
+  if (k % M != 0) return fail(NM_ERR_INVALID, "k=%lld is not a multiple of M=%d", (long long)k, M);
+  if (T <= 0 || T > INT32_MAX) return fail(NM_ERR_INVALID, "T must be in [1, 2^31-1] (got %lld)", (long long)T);
+  if (sms <= 0) return fail(NM_ERR_INVALID, "sms must be positive");
+  nm_handle h;  // the shape fields nm_compress derives; no device memory
+  h.n_out = n_out;
+  h.k = k;
+  h.N = N;
+  h.M = M;
+  h.dt = (int)dt;
+  h.img = sp24 ? nm::IMG_SP24 : nm::IMG_DENSE;
+  h.n_kb = (int)((k + nm::kblock_elems(h.dt) - 1) / nm::kblock_elems(h.dt));
+  h.n_ct = (int)((n_out + nm::kRows - 1) / nm::kRows);
+  Capacity c;
+  for (int i = 0; i < 3; ++i) c.pair[i] = pair_clusters[i];
+  for (int S = 1; S <= nm::kMaxClusterSplit; ++S) c.stream[S] = stream_clusters[S - 1];
+  const nm::Plan p = plan_with(&h, T, sms, c);
   out->pair = p.pair;
   out->bn = p.bn;
   out->splits = p.splits;
