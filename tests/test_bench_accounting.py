@@ -1,6 +1,7 @@
 """bench.py's accounting on CPU: algorithmic bytes, the roofline point and the
 whole-job throughput, checked against numbers worked out by hand from the
-layer shapes (ViT-B at T = 12608)."""
+layer shapes (ViT-B at T = 12608); and the clock sampler's placement of its
+NVML readings around the timed region (against a stand-in for pynvml)."""
 import pytest
 
 import bench
@@ -61,3 +62,62 @@ def test_roofline_point_gather_uses_kept_work_on_the_dense_pipe():
 def test_whole_job_tops():
     # 4 steps of 1e12 dense-equivalent ops on 2 ranks in 10 ms: 800 TOPS
     assert bench.whole_job_tops(10**12, 4, 2, 10.0) == pytest.approx(800.0)
+
+
+class _FakeNvml:
+    """Stands in for pynvml: records whether each power reading happened inside
+    the sampler's timed region."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self):
+        self.sampler = None
+        self.power_inside = []
+        self.clock_reads = 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus):
+        return "gpu0"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.clock_reads += 1
+        return 1965 if self.clock_reads % 2 else 1800
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x4  # sw_power_cap
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        self.power_inside.append(bool(self.sampler and self.sampler._inside))
+        return 400_000  # mW
+
+
+def test_clock_sampler_reads_power_only_outside_the_timed_region(monkeypatch):
+    """Power readings through NVML while the GPU ran the step stretched the timed
+    region, so the sampler polls clocks and reasons inside it and reads the
+    power just before and just after."""
+    import sys
+    import time
+    import types
+
+    import bench
+
+    fake = _FakeNvml()
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    props = types.SimpleNamespace(pci_domain_id=0, pci_bus_id=0x1b, pci_device_id=0)
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda dev: props)
+    with bench.NvmlSampler(0) as s:
+        fake.sampler = s
+        s.mark_start()
+        time.sleep(0.03)
+        s.poke()
+        s.mark_end()
+    summary = s.summary()
+    assert fake.power_inside == [False, False]  # one reading before, one after the region
+    assert summary["samples_in_timed_region"] >= 2 and fake.clock_reads >= 2
+    assert summary["reasons"] == ["sw_power_cap"]
+    assert summary["sm_max_mhz"] == 1965 and summary["sm_min_mhz"] in (1800, 1965)
+    assert summary["power_w_max"] == 400.0
